@@ -1,0 +1,203 @@
+/*
+ * bitsmoe.h -- C ABI of the B200 (sm_100a) library for the decode-time hot
+ * path of BitsMoE's spectral MoE gate/up projection.
+ *
+ * The method (BitsMoE study-note page, "BitsMoE: Cost-Aware Bit Allocation In
+ * spectral Space for MoE LLM Quantization"):
+ *   - Methodology, first split: one projection's experts share an input basis
+ *     Phi (from an SVD of the stacked expert matrices), so W_e x = P_e (Phi^T x)
+ *     and z = Phi^T x is computed once per token and reused by every selected
+ *     expert.
+ *   - second split: W_e = sum_k a_{e,k} p_{e,k} phi_k^T with unit directions
+ *     p_{e,k}; a_{e,k} is the component's amplitude.
+ *   - Usage: each component is stored at a width b in {0,1,2,3,4,6,8,16};
+ *     0 drops it, 16 keeps it as fp16.
+ *   - Execution: components of equal width are grouped and packed by bit plane.
+ * Quantiser (not on the pages; mid-rise, one fp16 scale per component):
+ *   s = fp16(2 max|p| / (2^b - 1)),  q = clamp(floor(p / s + 2^(b-1)), 0, 2^b - 1),
+ *   w = s (q - (2^b - 1)/2).
+ * Forward, per routed (token t, slot j) with expert e = ids[t][j]:
+ *   Y_e[t][j][i] = sum_b [ sum_bit 2^bit sum_{k in G_b} c_k bit_{k,bit,i}
+ *                          - (2^b - 1)/2 sum_{k in G_b} c_k ]  (+ fp16 group),
+ *   c_k = a_{e,k} s_{e,k} z_{t,k};  Y_sum[t][i] = sum_j g[t][j] Y_e[t][j][i].
+ *
+ * Conventions for every call:
+ *   - Pointers marked "dev" are device pointers (cudaMalloc, torch tensors...),
+ *     "host" are host pointers.  The caller allocates and owns every buffer;
+ *     the library never allocates device memory and keeps no device state.
+ *     Plans are host objects the library allocates and bitsmoe_plan_free frees.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every device
+ *     call is asynchronous on that stream; only bitsmoe_read_status waits.
+ *   - Return 0 on success or a negative BITSMOE_E* code.  Argument errors are
+ *     found on the host before any launch.  Data errors found on the device
+ *     (non-finite component, bad scale, expert id out of range, ...) are OR-ed
+ *     into a caller-owned device int32 `status` word as BITSMOE_ST_* bits; the
+ *     affected outputs are zero; nothing traps.
+ *   - fp16 values are passed as uint16_t bit patterns; fp32 as float.
+ *   - All arrays are dense, row-major, with the shapes written beside them.
+ *
+ * Packed format v1 (the blob written by bitsmoe_pack; little-endian).  Blob =
+ * header (64 B) | directory (E x 64 B) | expert 0 | expert 1 | ... ;
+ * d_pad = roundup(d_out, 8).
+ *   header: u32 magic "BMOE" | u32 version 1 | u32 d_out | u32 d_pad | u32 E |
+ *           u32 r | u64 total bytes | u64 64 | u64 64+64E | 16 zero bytes.
+ *   directory entry e: u64 base (byte offset of expert e) | u64 bytes |
+ *           u32 group offset from base [7] | u16 count [8] | u32 0;
+ *           groups and counts in width order 16,8,6,4,3,2,1 (count[7] = width 0).
+ *   group b in {1,2,3,4,6,8}, n members in ascending k, np = roundup(n,32):
+ *           u16 idx[np] | u16 fp16 scale[np] | f32 amp[np] |
+ *           u32 planes[b][np/32][d_pad]; bit m of word [j][w][i] is bit j of
+ *           q for member 32w+m at row i (row i fastest, 128-bit loads read 4
+ *           rows).
+ *   group 16, np = roundup(n,8): u16 idx[np] | f32 amp[np] | u16 w16[np][d_pad].
+ *   Every padding byte (members >= n, rows >= d_out) is zero.
+ */
+#ifndef BITSMOE_H
+#define BITSMOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ---- */
+#define BITSMOE_OK 0
+#define BITSMOE_EINVAL (-1)  /* bad dimension, NULL or misaligned pointer */
+#define BITSMOE_EWIDTH (-2)  /* a width outside {0,1,2,3,4,6,8,16} */
+#define BITSMOE_ESIZE (-3)   /* a buffer smaller than required */
+#define BITSMOE_ECUDA (-4)   /* a CUDA launch or API error (text in bitsmoe_strerror) */
+#define BITSMOE_EFORMAT (-5) /* a blob header/directory that does not parse */
+#define BITSMOE_ENOMEM (-6)  /* host allocation of a plan failed */
+
+/* ---- device status bits ---- */
+#define BITSMOE_ST_NONFINITE 1   /* a non-finite component element (its q or w16 is 0) */
+#define BITSMOE_ST_BADSCALE 2    /* a scale that is negative, NaN or Inf (its q are 0) */
+#define BITSMOE_ST_BADEXPERT 4   /* a routed expert id outside [0, E): zero Y_e row, left out of Y_sum */
+#define BITSMOE_ST_TIMEOUT 8     /* a bounded device wait gave up; outputs of that call are invalid */
+#define BITSMOE_ST_PLANMISMATCH 16 /* device widths disagree with the plan's widths */
+
+typedef struct {
+    int32_t d_in;      /* input width of the projection (rows of Phi) */
+    int32_t d_out;     /* output width (rows of each W_e), >= 1 */
+    int32_t n_experts; /* E >= 1 */
+    int32_t rank;      /* r = number of spectral components, 1 <= r <= 65535 */
+    int32_t top_k;     /* experts per token, >= 1 */
+} bitsmoe_dims;
+
+typedef struct bitsmoe_plan bitsmoe_plan;
+
+/* Plan the packed layout of one projection from its widths.
+ * widths_host [E][r] uint8 in {0,1,2,3,4,6,8,16}.  On success *out holds a
+ * new plan (free it with bitsmoe_plan_free).  Errors: EINVAL (dims, NULL),
+ * EWIDTH, ENOMEM.  (Usage: the width set; Execution: grouping by width.) */
+int bitsmoe_pack_plan(const bitsmoe_dims *dims, const uint8_t *widths_host, bitsmoe_plan **out);
+
+/* Rebuild a plan from the first bitsmoe_plan_header_bytes() bytes of a saved
+ * blob (host copy) plus the two dims a blob does not store (d_in, top_k).
+ * Checks magic, version and every directory entry.  Errors: EINVAL, EFORMAT,
+ * ESIZE (n_bytes shorter than header + directory), ENOMEM. */
+int bitsmoe_plan_from_header(const void *header_host, uint64_t n_bytes, int32_t d_in, int32_t top_k,
+                             bitsmoe_plan **out);
+
+void bitsmoe_plan_free(bitsmoe_plan *plan);
+
+/* Total bytes of the blob (header + directory + all experts); 0 for NULL. */
+uint64_t bitsmoe_plan_blob_bytes(const bitsmoe_plan *plan);
+
+/* Bytes of header + directory (= 64 + 64 E); 0 for NULL. */
+uint64_t bitsmoe_plan_header_bytes(const bitsmoe_plan *plan);
+
+/* Copies the plan's dims to *out.  Errors: EINVAL. */
+int bitsmoe_plan_get_dims(const bitsmoe_plan *plan, bitsmoe_dims *out);
+
+/* Copies header + directory (bitsmoe_plan_header_bytes bytes) to host_out.
+ * Errors: EINVAL, ESIZE. */
+int bitsmoe_plan_write_header(const bitsmoe_plan *plan, void *host_out, uint64_t capacity);
+
+/* Per-component fp16 scale s = fp16(2 max_i |p_i| / (2^b - 1)) for widths
+ * 1..8 (IEEE fp32 divide, round-to-nearest-even to fp16); 0 for widths 0 and
+ * 16.  comps dev [E][r][d_out] f32, widths dev [E][r] u8 (same values as the
+ * plan's), scales dev [E][r] u16 (out).  A component with a non-finite element
+ * gets scale 0 and BITSMOE_ST_NONFINITE.  status dev int32 or NULL.
+ * Errors: EINVAL, ECUDA. */
+int bitsmoe_compute_scales(const bitsmoe_plan *plan, const float *comps, const uint8_t *widths,
+                           uint16_t *scales, int32_t *status, void *stream);
+
+/* Quantise and pack one projection into `blob` (dev, bitsmoe_plan_blob_bytes
+ * bytes, 16-byte aligned).  comps dev [E][r][d_out] f32 (unit directions
+ * p_{e,k}), widths dev [E][r] u8, scales dev [E][r] u16 (fp16 bits, from
+ * bitsmoe_compute_scales or the caller's own), amps dev [E][r] f32.  Every
+ * byte of the blob is written; the result is bit-exact with the format above.
+ * Data errors go to *status (dev int32 or NULL).  Errors: EINVAL, ECUDA.
+ * (Execution: grouping by width, bit-plane packing; Usage: 0 and 16.) */
+int bitsmoe_pack(const bitsmoe_plan *plan, const float *comps, const uint8_t *widths,
+                 const uint16_t *scales, const float *amps, void *blob, int32_t *status, void *stream);
+
+/* Test support: unpack every component of `blob` (dev) to q dev [E][r][d_out]
+ * u16 (the b-bit integer for widths 1..8, the raw fp16 bits for width 16, 0
+ * for width 0).  Errors: EINVAL, ECUDA. */
+int bitsmoe_unpack_q(const bitsmoe_plan *plan, const void *blob, uint16_t *q, void *stream);
+
+/* Shared projection Z[t][k] = sum_i PhiT[k][i] X[t][i] (first split: z =
+ * Phi^T x, once per token).  phi_t dev [r][d_in] fp16 (row k = phi_k),
+ * X dev [T][d_in] fp16, Z dev [T][r] f32 (out); fp32 accumulation.
+ * phi_t and X must be 16-byte aligned and d_in a multiple of 8.  T = 0 is a
+ * no-op.  Errors: EINVAL, ECUDA. */
+int bitsmoe_shared_proj(const uint16_t *phi_t, const uint16_t *X, float *Z, int32_t T, int32_t d_in,
+                        int32_t r, void *stream);
+
+/* Workspace bytes bitsmoe_expert_forward needs for T tokens. */
+uint64_t bitsmoe_expert_workspace_bytes(const bitsmoe_plan *plan, int32_t T);
+
+/* Routed expert forward of one projection from a packed blob.
+ *   blob dev (packed by bitsmoe_pack for `plan`), Z dev [T][r] f32,
+ *   topk_ids dev [T][top_k] int32, gate_w dev [T][top_k] f32 (applied as
+ *   given, not renormalised), Y_experts dev [T][top_k][d_out] f32 or NULL,
+ *   Y_sum dev [T][d_out] f32, workspace dev (>= bitsmoe_expert_workspace_bytes,
+ *   256-byte aligned; contents need no initialisation), status dev or NULL.
+ * Tokens that share an expert are grouped so each expert's planes are read
+ * once per call.  Errors: EINVAL, ESIZE, ECUDA. */
+int bitsmoe_expert_forward(const bitsmoe_plan *plan, const void *blob, const float *Z, const int32_t *topk_ids,
+                           const float *gate_w, int32_t T, float *Y_experts, float *Y_sum, void *workspace,
+                           uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* One projection's buffers for bitsmoe_layer_forward. */
+typedef struct {
+    const bitsmoe_plan *plan; /* host plan of `blob` */
+    const void *blob;         /* dev packed blob */
+    const uint16_t *phi_t;    /* dev [r][d_in] fp16 */
+    float *Z;                 /* dev [T][r] f32 out, or NULL (then kept in the workspace) */
+    float *Y_experts;         /* dev [T][top_k][d_out] f32 out, or NULL */
+    float *Y_sum;             /* dev [T][d_out] f32 out */
+} bitsmoe_proj_io;
+
+/* Workspace bytes bitsmoe_layer_forward needs for T tokens. */
+uint64_t bitsmoe_layer_workspace_bytes(const bitsmoe_plan *gate, const bitsmoe_plan *up, int32_t T);
+
+/* Gate and up projections of one spectral MoE layer for T tokens: z = Phi^T x
+ * for both projections, then the routed experts of both, then their routed
+ * sums.  X dev [T][d_in] fp16; topk_ids / gate_w as in bitsmoe_expert_forward
+ * (shared by both projections).  The two plans must agree on d_in and top_k.
+ * workspace dev (>= bitsmoe_layer_workspace_bytes, 256-byte aligned); calls
+ * that share a workspace must not overlap on the GPU.  Errors: EINVAL, ESIZE,
+ * ECUDA. */
+int bitsmoe_layer_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,
+                          const int32_t *topk_ids, const float *gate_w, int32_t T, void *workspace,
+                          uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* Waits for `stream`, then copies the device status word to *out_host.
+ * Errors: EINVAL, ECUDA. */
+int bitsmoe_read_status(const int32_t *status_dev, void *stream, int32_t *out_host);
+
+/* Static text for a return code (for ECUDA, the last CUDA error seen by this
+ * thread's last failing call). */
+const char *bitsmoe_strerror(int code);
+
+/* Library version: 100 * major + minor. */
+int bitsmoe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITSMOE_H */

@@ -1,0 +1,213 @@
+"""ctypes binding of libbitsmoe (include/bitsmoe.h), same names as the C calls.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch tensors on the GPU (device pointers are taken with
+``data_ptr()``); the stream defaults to torch's current stream.  If the shared
+library is missing the import of any call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbitsmoe.so")
+
+OK, EINVAL, EWIDTH, ESIZE, ECUDA, EFORMAT, ENOMEM = 0, -1, -2, -3, -4, -5, -6
+ST_NONFINITE, ST_BADSCALE, ST_BADEXPERT, ST_TIMEOUT, ST_PLANMISMATCH = 1, 2, 4, 8, 16
+
+# Every symbol include/bitsmoe.h declares.
+EXPORTS = (
+    "bitsmoe_pack_plan", "bitsmoe_plan_from_header", "bitsmoe_plan_free", "bitsmoe_plan_blob_bytes",
+    "bitsmoe_plan_header_bytes", "bitsmoe_plan_get_dims", "bitsmoe_plan_write_header", "bitsmoe_compute_scales",
+    "bitsmoe_pack", "bitsmoe_unpack_q", "bitsmoe_shared_proj", "bitsmoe_expert_workspace_bytes",
+    "bitsmoe_expert_forward", "bitsmoe_layer_workspace_bytes", "bitsmoe_layer_forward", "bitsmoe_read_status",
+    "bitsmoe_strerror", "bitsmoe_version",
+)
+
+
+class BitsMoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("rank", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+
+class ProjIO(ctypes.Structure):
+    _fields_ = [("plan", ctypes.c_void_p), ("blob", ctypes.c_void_p), ("phi_t", ctypes.c_void_p),
+                ("Z", ctypes.c_void_p), ("Y_experts", ctypes.c_void_p), ("Y_sum", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with mixed_precision_decode_b200.build.build()")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, u64, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int32
+        sig = {
+            "bitsmoe_pack_plan": ([ctypes.POINTER(Dims), vp, ctypes.POINTER(vp)], ctypes.c_int),
+            "bitsmoe_plan_from_header": ([vp, u64, i32, i32, ctypes.POINTER(vp)], ctypes.c_int),
+            "bitsmoe_plan_free": ([vp], None),
+            "bitsmoe_plan_blob_bytes": ([vp], u64),
+            "bitsmoe_plan_header_bytes": ([vp], u64),
+            "bitsmoe_plan_get_dims": ([vp, ctypes.POINTER(Dims)], ctypes.c_int),
+            "bitsmoe_plan_write_header": ([vp, vp, u64], ctypes.c_int),
+            "bitsmoe_compute_scales": ([vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "bitsmoe_pack": ([vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "bitsmoe_unpack_q": ([vp, vp, vp, vp], ctypes.c_int),
+            "bitsmoe_shared_proj": ([vp, vp, vp, i32, i32, i32, vp], ctypes.c_int),
+            "bitsmoe_expert_workspace_bytes": ([vp, i32], u64),
+            "bitsmoe_expert_forward": ([vp, vp, vp, vp, vp, i32, vp, vp, vp, u64, vp, vp], ctypes.c_int),
+            "bitsmoe_layer_workspace_bytes": ([vp, vp, i32], u64),
+            "bitsmoe_layer_forward": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, i32, vp, u64,
+                                       vp, vp], ctypes.c_int),
+            "bitsmoe_read_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+            "bitsmoe_strerror": ([ctypes.c_int], ctypes.c_char_p),
+            "bitsmoe_version": ([], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().bitsmoe_strerror(code).decode()
+
+
+def version() -> int:
+    return lib().bitsmoe_version()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise BitsMoEError(rc, what)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    return int(t)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+class Plan:
+    """Owns one bitsmoe_plan (host object describing one projection's blob)."""
+
+    def __init__(self, handle: int):
+        self._h = ctypes.c_void_p(handle)
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._h
+
+    def __del__(self):
+        if getattr(self, "_h", None) is not None and self._h.value and _lib is not None:
+            _lib.bitsmoe_plan_free(self._h)
+            self._h = None
+
+    @property
+    def blob_bytes(self) -> int:
+        return int(lib().bitsmoe_plan_blob_bytes(self._h))
+
+    @property
+    def header_bytes(self) -> int:
+        return int(lib().bitsmoe_plan_header_bytes(self._h))
+
+    @property
+    def dims(self) -> Dims:
+        d = Dims()
+        _check(lib().bitsmoe_plan_get_dims(self._h, ctypes.byref(d)), "plan_get_dims")
+        return d
+
+    def header(self) -> np.ndarray:
+        out = np.zeros(self.header_bytes, np.uint8)
+        _check(lib().bitsmoe_plan_write_header(self._h, out.ctypes.data, out.size), "plan_write_header")
+        return out
+
+
+def pack_plan(d_in: int, d_out: int, n_experts: int, rank: int, top_k: int, widths) -> Plan:
+    w = np.ascontiguousarray(widths.cpu().numpy() if isinstance(widths, torch.Tensor) else widths, dtype=np.uint8)
+    d = Dims(d_in, d_out, n_experts, rank, top_k)
+    h = ctypes.c_void_p()
+    _check(lib().bitsmoe_pack_plan(ctypes.byref(d), w.ctypes.data, ctypes.byref(h)), "pack_plan")
+    return Plan(h.value)
+
+
+def plan_from_header(header, d_in: int, top_k: int) -> Plan:
+    hb = np.ascontiguousarray(header.cpu().numpy() if isinstance(header, torch.Tensor) else header, dtype=np.uint8)
+    h = ctypes.c_void_p()
+    _check(lib().bitsmoe_plan_from_header(hb.ctypes.data, hb.size, d_in, top_k, ctypes.byref(h)), "plan_from_header")
+    return Plan(h.value)
+
+
+def compute_scales(plan: Plan, comps, widths, scales, status=None, stream=None):
+    _check(lib().bitsmoe_compute_scales(plan.handle, _ptr(comps), _ptr(widths), _ptr(scales), _ptr(status),
+                                        _stream(stream)), "compute_scales")
+
+
+def pack(plan: Plan, comps, widths, scales, amps, blob, status=None, stream=None):
+    _check(lib().bitsmoe_pack(plan.handle, _ptr(comps), _ptr(widths), _ptr(scales), _ptr(amps), _ptr(blob),
+                              _ptr(status), _stream(stream)), "pack")
+
+
+def unpack_q(plan: Plan, blob, q, stream=None):
+    _check(lib().bitsmoe_unpack_q(plan.handle, _ptr(blob), _ptr(q), _stream(stream)), "unpack_q")
+
+
+def shared_proj(phi_t, X, Z, T: int, d_in: int, r: int, stream=None):
+    _check(lib().bitsmoe_shared_proj(_ptr(phi_t), _ptr(X), _ptr(Z), T, d_in, r, _stream(stream)), "shared_proj")
+
+
+def expert_workspace_bytes(plan: Plan, T: int) -> int:
+    return int(lib().bitsmoe_expert_workspace_bytes(plan.handle, T))
+
+
+def expert_forward(plan: Plan, blob, Z, topk_ids, gate_w, T: int, Y_experts, Y_sum, workspace, workspace_bytes: int,
+                   status=None, stream=None):
+    _check(lib().bitsmoe_expert_forward(plan.handle, _ptr(blob), _ptr(Z), _ptr(topk_ids), _ptr(gate_w), T,
+                                        _ptr(Y_experts), _ptr(Y_sum), _ptr(workspace), workspace_bytes,
+                                        _ptr(status), _stream(stream)), "expert_forward")
+
+
+def layer_workspace_bytes(plan_gate: Plan, plan_up: Plan, T: int) -> int:
+    return int(lib().bitsmoe_layer_workspace_bytes(plan_gate.handle, plan_up.handle, T))
+
+
+def proj_io(plan: Plan, blob, phi_t, Y_sum, Z=None, Y_experts=None) -> ProjIO:
+    return ProjIO(plan.handle.value, _ptr(blob), _ptr(phi_t), _ptr(Z), _ptr(Y_experts), _ptr(Y_sum))
+
+
+def layer_forward(gate: ProjIO, up: ProjIO, X, topk_ids, gate_w, T: int, workspace, workspace_bytes: int,
+                  status=None, stream=None):
+    _check(lib().bitsmoe_layer_forward(ctypes.byref(gate), ctypes.byref(up), _ptr(X), _ptr(topk_ids), _ptr(gate_w),
+                                       T, _ptr(workspace), workspace_bytes, _ptr(status), _stream(stream)),
+           "layer_forward")
+
+
+def read_status(status, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check(lib().bitsmoe_read_status(_ptr(status), _stream(stream), ctypes.byref(out)), "read_status")
+    return int(out.value)

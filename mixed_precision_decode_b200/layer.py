@@ -1,0 +1,87 @@
+"""User-facing objects over the C ABI: a packed projection and a spectral MoE
+gate/up layer.  torch provides device memory and streams; every computation
+is a libbitsmoe kernel."""
+from __future__ import annotations
+
+import torch
+
+from . import bitsmoe as B
+
+
+class PackedProjection:
+    """One projection (gate or up) of a spectral MoE layer, packed on the GPU.
+
+    phi_t [r][d_in] fp16 (rows phi_k, kept unquantised), blob = the format-v1
+    bit-plane blob of the expert directions, plan = its host descriptor."""
+
+    def __init__(self, plan: B.Plan, blob: torch.Tensor, phi_t: torch.Tensor):
+        self.plan, self.blob, self.phi_t = plan, blob, phi_t
+        d = plan.dims
+        self.d_in, self.d_out, self.n_experts, self.rank, self.top_k = d.d_in, d.d_out, d.n_experts, d.rank, d.top_k
+
+    @classmethod
+    def from_factors(cls, phi_t: torch.Tensor, amps: torch.Tensor, comps: torch.Tensor, widths: torch.Tensor,
+                     top_k: int, scales: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                     stream=None) -> "PackedProjection":
+        """Quantise and pack unit directions comps [E][r][d_out] (f32, on the GPU) at
+        widths [E][r] (u8) with amplitudes amps [E][r] (f32)."""
+        E, r, d_out = comps.shape
+        d_in = phi_t.shape[1]
+        dev = comps.device
+        plan = B.pack_plan(d_in, d_out, E, r, top_k, widths.cpu())
+        w_dev = widths.to(dev, torch.uint8).contiguous()
+        if scales is None:
+            scales = torch.empty((E, r), dtype=torch.int16, device=dev)
+            B.compute_scales(plan, comps, w_dev, scales, status, stream)
+        blob = torch.empty(plan.blob_bytes, dtype=torch.uint8, device=dev)
+        B.pack(plan, comps.contiguous(), w_dev, scales.contiguous(), amps.contiguous(), blob, status, stream)
+        return cls(plan, blob, phi_t.contiguous())
+
+    def expert_bytes_touched(self, experts) -> int:
+        """Packed bytes (planes + per-component metadata, padding included) of the given experts."""
+        h = self.plan.header()
+        tot = 0
+        for e in experts:
+            d = h[64 + 64 * int(e): 128 + 64 * int(e)]
+            tot += int(d[8:16].view("uint64")[0])
+        return tot
+
+
+class SpectralMoELayer:
+    """Gate and up projections of one MoE layer in shared-spectral form."""
+
+    def __init__(self, gate: PackedProjection, up: PackedProjection):
+        assert gate.d_in == up.d_in and gate.top_k == up.top_k and gate.n_experts == up.n_experts
+        self.gate, self.up = gate, up
+        self._ws = {}
+
+    def workspace(self, T: int) -> torch.Tensor:
+        n = B.layer_workspace_bytes(self.gate.plan, self.up.plan, T)
+        ws = self._ws.get(T)
+        if ws is None or ws.numel() < n:
+            ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.gate.blob.device)
+            self._ws[T] = ws
+        return ws
+
+    def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, gate_w: torch.Tensor, out: dict | None = None,
+                want_experts: bool = False, want_z: bool = False, status: torch.Tensor | None = None,
+                stream=None) -> dict:
+        """x [T][d_in] fp16, topk_ids [T][top_k] int32, gate_w [T][top_k] f32 (all on the GPU).
+        Returns Y_sum_gate / Y_sum_up [T][d_out] f32 (and Y_experts_* / Z_* on request)."""
+        T = x.shape[0]
+        dev = x.device
+        if out is None:
+            out = {}
+            for name, p in (("gate", self.gate), ("up", self.up)):
+                out[f"Y_sum_{name}"] = torch.empty((T, p.d_out), dtype=torch.float32, device=dev)
+                if want_experts:
+                    out[f"Y_experts_{name}"] = torch.empty((T, p.top_k, p.d_out), dtype=torch.float32, device=dev)
+                if want_z:
+                    out[f"Z_{name}"] = torch.empty((T, p.rank), dtype=torch.float32, device=dev)
+        ios = []
+        for name, p in (("gate", self.gate), ("up", self.up)):
+            ios.append(B.proj_io(p.plan, p.blob, p.phi_t, out[f"Y_sum_{name}"], out.get(f"Z_{name}"),
+                                 out.get(f"Y_experts_{name}")))
+        ws = self.workspace(T)
+        B.layer_forward(ios[0], ios[1], x, topk_ids, gate_w, T, ws, ws.numel(), status, stream)
+        return out

@@ -106,6 +106,8 @@ def make_projection(cfg: LayerConfig, gen: torch.Generator, device, experts=None
     """One projection's factors: phi_t [r][d_in] fp16, amps [E][r] f32,
     comps [E][r][d_out] f32 (unit rows), widths [E][r] u8."""
     d_in, d_out, E, r = cfg.d_in, cfg.d_out, cfg.n_experts, cfg.rank
+    if r > d_in:
+        raise ValueError(f"rank {r} > d_in {d_in}: an orthonormal basis of the input space has at most d_in columns")
     A = torch.randn((d_in, r), generator=gen, device=device, dtype=torch.float32)
     Q, _ = torch.linalg.qr(A)
     phi_t = Q.T.contiguous().to(torch.float16)

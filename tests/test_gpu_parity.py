@@ -1,0 +1,154 @@
+"""CUDA path vs the oracle, element by element, on the same seeded inputs.
+
+Bit-exact: scales, the packed blob (every byte, padding included) and the
+unpacked integers.  Within 2e-3 max relative error per output vector (the
+bound stated for fp32 accumulation against the fp64 oracle): Z, Y_e, Y_sum.
+Small cases are compared in full; full-size Qwen3-30B-A3B- and Mixtral-shaped
+layers on sampled experts and tokens, in the launch configuration the
+benchmark uses."""
+import numpy as np
+import pytest
+import torch
+
+from cases import FULL, SMALL, TOL, expert_section, get_case, rel_err, x_bits
+from mixed_precision_decode_b200 import bitsmoe as B
+
+pytestmark = pytest.mark.gpu
+
+ALL = list(SMALL) + list(FULL)
+
+
+def _sample_experts(case, n=4):
+    E = case.cfg.n_experts
+    if case.cfg.name in SMALL:
+        return list(range(E))
+    ids = case.ids.cpu().numpy()
+    pick = {0, E - 1, int(ids[0, 0])}
+    if case.cfg.d_out * case.cfg.rank < 4_000_000:
+        pick.add(E // 2)
+    return sorted(pick)
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_scales_bitexact(name, orc):
+    case = get_case(name)
+    for proj in ("gate", "up"):
+        pk = case.proj[proj]
+        h = case.host[proj]
+        E, r = h["widths"].shape
+        scales = torch.empty((E, r), dtype=torch.int16, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        B.compute_scales(pk.plan, h["comps_dev"], torch.as_tensor(h["widths"], device="cuda"), scales, st)
+        ex = _sample_experts(case)
+        _, ref, ost = case.oracle_blob(orc, proj, ex)
+        got = scales.cpu().numpy().view(np.uint16)[ex]
+        assert np.array_equal(got, ref)
+        assert B.read_status(st) == 0 and ost == 0
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_pack_bitexact(name, orc):
+    case = get_case(name)
+    assert B.read_status(case.status) == 0
+    for proj in ("gate", "up"):
+        gpu = case.gpu_blob(proj)
+        plan = case.proj[proj].plan
+        assert gpu.size == plan.blob_bytes
+        assert np.array_equal(gpu[:plan.header_bytes], plan.header())
+        ex = _sample_experts(case)
+        ref, _, _ = case.oracle_blob(orc, proj, ex)
+        if len(ex) == case.cfg.n_experts:
+            assert np.array_equal(gpu, ref), np.flatnonzero(gpu != ref)[:8]
+        else:
+            for j, e in enumerate(ex):
+                a, b = expert_section(gpu, e), expert_section(ref, j)
+                assert a.size == b.size and np.array_equal(a, b), (proj, e, np.flatnonzero(a != b)[:8])
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_unpack_bitexact(name, orc):
+    case = get_case(name)
+    for proj in ("gate", "up"):
+        pk = case.proj[proj]
+        E, r = case.host[proj]["widths"].shape
+        d_out = case.cfg.d_out
+        q = torch.empty((E, r, d_out), dtype=torch.int16, device="cuda")
+        B.unpack_q(pk.plan, pk.blob, q)
+        ex = _sample_experts(case)
+        ref_blob, _, _ = case.oracle_blob(orc, proj, ex)
+        qref, wref, _, _ = orc.unpack(ref_blob)
+        got = q[torch.as_tensor(ex, device="cuda")].cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, qref)
+        del q
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_shared_proj(name, orc):
+    case = get_case(name)
+    T = case.cfg.tokens
+    for proj in ("gate", "up"):
+        pk = case.proj[proj]
+        Z = torch.empty((T, case.cfg.rank), dtype=torch.float32, device="cuda")
+        B.shared_proj(pk.phi_t, case.x, Z, T, case.cfg.d_in, case.cfg.rank)
+        ref = orc.shared_proj(case.host[proj]["phi_t"], x_bits(case))
+        assert rel_err(Z.cpu().numpy(), ref) <= TOL
+
+
+def _tokens(case):
+    T = case.cfg.tokens
+    if case.cfg.name in SMALL or T <= 4:
+        return list(range(T))
+    return [0, T // 3, T - 1] if case.cfg.d_out * case.cfg.rank < 4_000_000 else [0, T - 1]
+
+
+def _oracle_tokens(case, orc, proj, toks, Z):
+    """Oracle Y_e / Y_sum for the given tokens, on a blob of just their experts."""
+    ids = case.ids.cpu().numpy()[toks]
+    g = case.gate_w.cpu().numpy()[toks]
+    ex = sorted(set(int(v) for v in ids.ravel()))
+    remap = {e: j for j, e in enumerate(ex)}
+    blob, _, _ = case.oracle_blob(orc, proj, ex)
+    rid = np.vectorize(remap.get)(ids).astype(np.int32)
+    Ye, Ys, st = orc.expert_forward(blob, Z, rid, g)
+    assert st == 0
+    return Ye, Ys
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_expert_forward(name, orc):
+    """The expert step alone: both sides take the CUDA path's Z as input."""
+    case = get_case(name)
+    T, K, d_out, r = case.cfg.tokens, case.cfg.top_k, case.cfg.d_out, case.cfg.rank
+    toks = _tokens(case)
+    for proj in ("gate", "up"):
+        pk = case.proj[proj]
+        Z = torch.empty((T, r), dtype=torch.float32, device="cuda")
+        B.shared_proj(pk.phi_t, case.x, Z, T, case.cfg.d_in, r)
+        Ye = torch.empty((T, K, d_out), dtype=torch.float32, device="cuda")
+        Ys = torch.empty((T, d_out), dtype=torch.float32, device="cuda")
+        n = B.expert_workspace_bytes(pk.plan, T)
+        ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        B.expert_forward(pk.plan, pk.blob, Z, case.ids, case.gate_w, T, Ye, Ys, ws, n, st)
+        assert B.read_status(st) == 0
+        Zh = Z.cpu().numpy().astype(np.float64)[toks]
+        Ye_ref, Ys_ref = _oracle_tokens(case, orc, proj, toks, Zh)
+        assert rel_err(Ye.cpu().numpy()[toks], Ye_ref) <= TOL
+        assert rel_err(Ys.cpu().numpy()[toks], Ys_ref) <= TOL
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_layer_forward(name, orc):
+    """End to end through the layer call (the fused path where it applies)
+    against the oracle's own z = Phi^T x and expert forward."""
+    case = get_case(name)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = case.layer.forward(case.x, case.ids, case.gate_w, want_experts=True, want_z=True, status=st)
+    assert B.read_status(st) == 0
+    toks = _tokens(case)
+    for proj in ("gate", "up"):
+        Zref = orc.shared_proj(case.host[proj]["phi_t"], x_bits(case))
+        assert rel_err(out[f"Z_{proj}"].cpu().numpy(), Zref) <= TOL
+        Ye_ref, Ys_ref = _oracle_tokens(case, orc, proj, toks, Zref[toks])
+        assert rel_err(out[f"Y_experts_{proj}"].cpu().numpy()[toks], Ye_ref) <= TOL
+        assert rel_err(out[f"Y_sum_{proj}"].cpu().numpy()[toks], Ys_ref) <= TOL
