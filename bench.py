@@ -355,7 +355,7 @@ def run_ours(args, dist):
 
     peak, peak_kind = load_peak()
     achieved = alg["total"] / step_s / 1e9
-    launches_per_step = kernels_per_step(T)
+    launches_per_step = kernels_per_step(wl)
 
     # end to end through the public API: pinned host inputs -> device, forward, outputs -> pinned host
     e2e = None
@@ -367,7 +367,7 @@ def run_ours(args, dist):
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded random factors of the layer's shape; no checkpoint)",
         "config": workload_config(cfg, T, args.layers, wl.blob_bytes_total(), alg["total"]),
-        "roofline": {"bound": "hbm", "kernel": dominant_kernel(T), "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": dominant_kernel(launches_per_step), "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                      "algorithmic_bytes_per_launch": alg["total"], "bytes_breakdown": {k: alg[k] for k in
                                                                                        ("phi", "planes", "meta", "act")},
@@ -386,25 +386,15 @@ def run_ours(args, dist):
         print(json.dumps(line), flush=True)
 
 
-def kernels_per_step(T: int) -> int:
+def kernels_per_step(wl) -> int:
     from mixed_precision_decode_b200 import bitsmoe as B
-    return B.lib().bitsmoe_version() and (1 if T == 1 and fused_t1_available() else 7)
+    L = wl.layers[0]
+    return B.layer_launches(L.gate.plan, L.up.plan, wl.cfg.tokens)
 
 
-def fused_t1_available() -> bool:
-    return os.environ.get("BITSMOE_T1_FUSED", "1") != "0" and _probe_fused()
-
-
-def _probe_fused() -> bool:
-    try:
-        from mixed_precision_decode_b200 import bitsmoe as B
-        return bool(B.lib().bitsmoe_version() >= 101)
-    except Exception:
-        return False
-
-
-def dominant_kernel(T: int) -> str:
-    return "k_layer_t1" if T == 1 and fused_t1_available() else "whole step (k_route, k_shared_proj x2, k_expert_general x2, k_combine x2)"
+def dominant_kernel(n_launches: int) -> str:
+    return "k_layer_t1 (fused single-token layer)" if n_launches == 1 else \
+        "whole step: k_route, k_shared_proj x2, k_expert_general x2, k_combine x2"
 
 
 def run_e2e(wl, cfg, T, n, dist):

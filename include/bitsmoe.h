@@ -175,13 +175,23 @@ typedef struct {
 /* Workspace bytes bitsmoe_layer_forward needs for T tokens. */
 uint64_t bitsmoe_layer_workspace_bytes(const bitsmoe_plan *gate, const bitsmoe_plan *up, int32_t T);
 
+/* Number of kernels one bitsmoe_layer_forward call launches for T tokens with
+ * these plans: 1 when the fused single-token path applies (T = 1 and the
+ * shapes fit one CTA per SM), else 7 (routing groups, then per projection the
+ * shared projection, the experts and the routed combine); 0 for T = 0.
+ * Errors: EINVAL. */
+int bitsmoe_layer_launches(const bitsmoe_plan *gate, const bitsmoe_plan *up, int32_t T);
+
 /* Gate and up projections of one spectral MoE layer for T tokens: z = Phi^T x
  * for both projections, then the routed experts of both, then their routed
  * sums.  X dev [T][d_in] fp16; topk_ids / gate_w as in bitsmoe_expert_forward
  * (shared by both projections).  The two plans must agree on d_in and top_k.
- * workspace dev (>= bitsmoe_layer_workspace_bytes, 256-byte aligned); calls
- * that share a workspace must not overlap on the GPU.  Errors: EINVAL, ESIZE,
- * ECUDA. */
+ * workspace dev (>= bitsmoe_layer_workspace_bytes, 256-byte aligned) must be
+ * zero-filled once before its first use: its head holds counters of the fused
+ * single-token path that every call leaves ready for the next one (after a
+ * BITSMOE_ST_TIMEOUT status, zero it again).  Calls that share a workspace
+ * must not overlap on the GPU.  With T = 1 the routed sum is formed in slot
+ * order, so results do not depend on timing.  Errors: EINVAL, ESIZE, ECUDA. */
 int bitsmoe_layer_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,
                           const int32_t *topk_ids, const float *gate_w, int32_t T, void *workspace,
                           uint64_t workspace_bytes, int32_t *status, void *stream);

@@ -23,7 +23,8 @@ EXPORTS = (
     "bitsmoe_pack_plan", "bitsmoe_plan_from_header", "bitsmoe_plan_free", "bitsmoe_plan_blob_bytes",
     "bitsmoe_plan_header_bytes", "bitsmoe_plan_get_dims", "bitsmoe_plan_write_header", "bitsmoe_compute_scales",
     "bitsmoe_pack", "bitsmoe_unpack_q", "bitsmoe_shared_proj", "bitsmoe_expert_workspace_bytes",
-    "bitsmoe_expert_forward", "bitsmoe_layer_workspace_bytes", "bitsmoe_layer_forward", "bitsmoe_read_status",
+    "bitsmoe_expert_forward", "bitsmoe_layer_workspace_bytes", "bitsmoe_layer_launches", "bitsmoe_layer_forward",
+    "bitsmoe_read_status",
     "bitsmoe_strerror", "bitsmoe_version",
 )
 
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "bitsmoe_expert_workspace_bytes": ([vp, i32], u64),
             "bitsmoe_expert_forward": ([vp, vp, vp, vp, vp, i32, vp, vp, vp, u64, vp, vp], ctypes.c_int),
             "bitsmoe_layer_workspace_bytes": ([vp, vp, i32], u64),
+            "bitsmoe_layer_launches": ([vp, vp, i32], ctypes.c_int),
             "bitsmoe_layer_forward": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, i32, vp, u64,
                                        vp, vp], ctypes.c_int),
             "bitsmoe_read_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
@@ -194,6 +196,13 @@ def expert_forward(plan: Plan, blob, Z, topk_ids, gate_w, T: int, Y_experts, Y_s
 
 def layer_workspace_bytes(plan_gate: Plan, plan_up: Plan, T: int) -> int:
     return int(lib().bitsmoe_layer_workspace_bytes(plan_gate.handle, plan_up.handle, T))
+
+
+def layer_launches(plan_gate: Plan, plan_up: Plan, T: int) -> int:
+    n = int(lib().bitsmoe_layer_launches(plan_gate.handle, plan_up.handle, T))
+    if n < 0:
+        raise BitsMoEError(n, "layer_launches")
+    return n
 
 
 def proj_io(plan: Plan, blob, phi_t, Y_sum, Z=None, Y_experts=None) -> ProjIO:

@@ -59,7 +59,8 @@ class SpectralMoELayer:
         n = B.layer_workspace_bytes(self.gate.plan, self.up.plan, T)
         ws = self._ws.get(T)
         if ws is None or ws.numel() < n:
-            ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.gate.blob.device)
+            # zero-filled once: its head keeps the fused path's counters between calls
+            ws = torch.zeros(max(n, 256), dtype=torch.uint8, device=self.gate.blob.device)
             self._ws[T] = ws
         return ws
 

@@ -106,3 +106,16 @@ def get_case(name: str) -> Case:
 
 def x_bits(case: Case) -> np.ndarray:
     return case.x.cpu().numpy().view(np.uint16)
+
+
+def oracle_tokens(case: Case, orc, proj: str, toks, Z, ids=None, gate_w=None):
+    """Oracle Y_e / Y_sum for the given tokens, on a blob of just their experts."""
+    ids = (case.ids if ids is None else ids).cpu().numpy()[toks]
+    g = (case.gate_w if gate_w is None else gate_w).cpu().numpy()[toks]
+    ex = sorted(set(int(v) for v in ids.ravel()))
+    remap = {e: j for j, e in enumerate(ex)}
+    blob, _, _ = case.oracle_blob(orc, proj, ex)
+    rid = np.vectorize(remap.get)(ids).astype(np.int32)
+    Ye, Ys, st = orc.expert_forward(blob, Z, rid, g)
+    assert st == 0
+    return Ye, Ys

@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from cases import FULL, SMALL, TOL, expert_section, get_case, rel_err, x_bits
+from cases import FULL, SMALL, TOL, expert_section, get_case, oracle_tokens, rel_err, x_bits
 from mixed_precision_decode_b200 import bitsmoe as B
 
 pytestmark = pytest.mark.gpu
@@ -102,16 +102,7 @@ def _tokens(case):
 
 
 def _oracle_tokens(case, orc, proj, toks, Z):
-    """Oracle Y_e / Y_sum for the given tokens, on a blob of just their experts."""
-    ids = case.ids.cpu().numpy()[toks]
-    g = case.gate_w.cpu().numpy()[toks]
-    ex = sorted(set(int(v) for v in ids.ravel()))
-    remap = {e: j for j, e in enumerate(ex)}
-    blob, _, _ = case.oracle_blob(orc, proj, ex)
-    rid = np.vectorize(remap.get)(ids).astype(np.int32)
-    Ye, Ys, st = orc.expert_forward(blob, Z, rid, g)
-    assert st == 0
-    return Ye, Ys
+    return oracle_tokens(case, orc, proj, toks, Z)
 
 
 @pytest.mark.parametrize("name", ALL)
