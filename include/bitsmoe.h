@@ -196,6 +196,26 @@ int bitsmoe_layer_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up
                           const int32_t *topk_ids, const float *gate_w, int32_t T, void *workspace,
                           uint64_t workspace_bytes, int32_t *status, void *stream);
 
+/* Single-token layer forward (T = 1) that allocates nothing: the same fused
+ * kernel as bitsmoe_layer_forward, with its scratch taken from one fixed 1 MiB
+ * array that the library keeps in device memory (every GPU that loads the
+ * library holds it until the process exits).  The BitsMoE pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory or hand out a workspace -- a serving runtime that owns all device
+ * memory through its own pool, a plugin that is only given its input and
+ * output buffers, or a decode loop that must not call cudaMalloc because it
+ * synchronises the device and cannot be recorded into a CUDA graph.
+ *   gate, up, X, topk_ids, gate_w, status: as in bitsmoe_layer_forward with
+ *   T = 1 (topk_ids / gate_w hold one row of top_k entries).
+ * The first call on each device looks up the array's device address; make
+ * that first call before any stream capture.  Every call clears the array's
+ * counters and then uses it, so calls that overlap on the GPU (two streams,
+ * two host threads) race and must be serialised by the caller.
+ * Errors: EINVAL (dims, NULL or misaligned pointers), ESIZE (shapes the
+ * single-launch kernel cannot hold, or scratch beyond 1 MiB), ECUDA. */
+int bitsmoe_layer_forward_t1_noalloc(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,
+                                     const int32_t *topk_ids, const float *gate_w, int32_t *status, void *stream);
+
 /* Waits for `stream`, then copies the device status word to *out_host.
  * Errors: EINVAL, ECUDA. */
 int bitsmoe_read_status(const int32_t *status_dev, void *stream, int32_t *out_host);

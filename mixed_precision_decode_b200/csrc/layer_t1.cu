@@ -19,6 +19,7 @@
 // bits.  The routed sum is done by the last CTA to finish each row block, in
 // slot order, so results do not depend on timing.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -663,3 +664,71 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
 }
 
 }  // namespace bitsmoe
+
+// ---------------------------------------------------------------------------
+// Single-token layer forward with library-owned scratch, for callers that
+// cannot allocate device memory.  The scratch (the fused kernel's grid-barrier
+// counter, row-block counters, z of both projections and the weighted rows of
+// the routed sum) lives in one fixed static device array instead of a
+// caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace bitsmoe {
+
+constexpr uint64_t kNoAllocScratchBytes = 1ull << 20;  // 1 MiB, held by every GPU that loads the library
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 256;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kNoAllocMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  (In host code the array's name is only a host-side handle.)
+static int noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return set_cuda_error(e);
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return BITSMOE_EINVAL;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return set_cuda_error(e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return BITSMOE_OK;
+}
+
+}  // namespace bitsmoe
+
+BITSMOE_API int bitsmoe_layer_forward_t1_noalloc(const bitsmoe_proj_io* gate, const bitsmoe_proj_io* up,
+                                                 const uint16_t* X, const int32_t* topk_ids, const float* gate_w,
+                                                 int32_t* status, void* stream) {
+    using namespace bitsmoe;
+    if (!gate || !up || !gate->plan || !up->plan || !X || !topk_ids || !gate_w) return BITSMOE_EINVAL;
+    const bitsmoe_proj_io* io[2] = {gate, up};
+    const bitsmoe_plan *pg = gate->plan, *pu = up->plan;
+    if (pg->dims.d_in != pu->dims.d_in || pg->dims.top_k != pu->dims.top_k ||
+        pg->dims.n_experts != pu->dims.n_experts || pg->dims.d_in % 8)
+        return BITSMOE_EINVAL;
+    for (int j = 0; j < 2; j++) {
+        if (!io[j]->blob || !io[j]->phi_t || !io[j]->Y_sum) return BITSMOE_EINVAL;
+        if ((uintptr_t)io[j]->blob % 16 || (uintptr_t)io[j]->phi_t % 16) return BITSMOE_EINVAL;
+    }
+    if ((uintptr_t)X % 16) return BITSMOE_EINVAL;
+    // shapes the single-launch kernel cannot hold, or whose scratch exceeds the array
+    const uint64_t head = layer_fused_t1_reserved(pg, pu);
+    const uint64_t rest = layer_fused_t1_workspace(pg, pu);
+    if (head == 0 || rest == 0 || head + rest > kNoAllocScratchBytes) return BITSMOE_ESIZE;
+    void* scratch = nullptr;
+    int rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    cudaStream_t s = (cudaStream_t)stream;
+    // the counters must start at zero; the array keeps whatever the last call left
+    cudaError_t e = cudaMemsetAsync(scratch, 0, head, s);
+    if (e != cudaSuccess) return set_cuda_error(e);
+    bool used = false;
+    rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, scratch, head + rest, status, s, &used);
+    if (rc) return rc;
+    return used ? BITSMOE_OK : BITSMOE_ESIZE;
+}
