@@ -53,6 +53,12 @@ __host__ __device__ inline uint64_t group_bytes(int b, uint64_t n, uint64_t d_pa
     return 8 * np + 4 * (uint64_t)b * (np / 32) * d_pad;
 }
 
+// Word index of plane word [tile i/32][plane j][word w][row i%32] inside a
+// group's planes (32-row tiles; W = words per plane, b = planes).
+__host__ __device__ inline uint64_t plane_word(uint32_t j, uint32_t w, uint32_t W, int b, uint32_t i) {
+    return ((((uint64_t)(i >> 5) * (uint64_t)b + j) * W + w) << 5) + (i & 31u);
+}
+
 // Directory entry of one expert, decoded.
 struct DirEntry {
     uint64_t base;          // byte offset of the expert's data in the blob
@@ -79,7 +85,7 @@ struct QGroup {
     const uint16_t* idx;
     const uint16_t* scale;
     const float* amp;
-    const uint32_t* planes;  // [b][W][d_pad]
+    const uint32_t* planes;  // [d_pad/32][b][W][32]
     uint32_t n, np, W;
 };
 __device__ inline QGroup qgroup(const uint8_t* blob, const DirEntry& d, int g) {

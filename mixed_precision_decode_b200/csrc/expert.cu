@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kExThreads) k_expert_general(const uint8_t* __
                     const uint32_t W = np / 32;
                     for (uint32_t w = m0 / 32; w < m1 / 32; w++) {
                         for (int pb = 0; pb < b; pb++) {
-                            uint32_t word = planes[((uint64_t)pb * W + w) * d_pad + i];
+                            uint32_t word = planes[plane_word(pb, w, W, b, i)];
                             const float wt = (float)(1u << pb);
                             float part[kTC];
 #pragma unroll

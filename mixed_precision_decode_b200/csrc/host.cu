@@ -33,7 +33,7 @@ static bool dims_ok(const bitsmoe_dims* d) {
 // Fills sizes, the header image and the derived launch bounds from counts.
 static int finish_plan(bitsmoe_plan* p) {
     const int E = p->dims.n_experts;
-    p->d_pad = (uint32_t)roundup((uint64_t)p->dims.d_out, 8);
+    p->d_pad = (uint32_t)roundup((uint64_t)p->dims.d_out, 32);
     p->header_bytes = kHeaderBytes + kDirEntryBytes * (uint64_t)E;
     p->header = (uint8_t*)calloc(p->header_bytes, 1);
     if (!p->header) return BITSMOE_ENOMEM;

@@ -25,7 +25,10 @@
 
 namespace bitsmoe {
 
-constexpr int kT1Threads = 512;
+#ifndef BITSMOE_T1_THREADS
+#define BITSMOE_T1_THREADS 512
+#endif
+constexpr int kT1Threads = BITSMOE_T1_THREADS;  // threads per CTA of the fused kernel
 constexpr int kT1Warps = kT1Threads / 32;
 constexpr int kRB = 32;            // rows per task (one per lane)
 constexpr int kMaxUnitsPerCta = 8;
@@ -60,7 +63,7 @@ struct T1Params {
     int n16_max;        // fp16 members per unit (upper bound)
     // shared-memory layout (byte offsets)
     uint32_t sm_x, sm_a, sm_planes, sm_meta, sm_end;
-    uint32_t a_z, a_tab, a_part, a_c16, a_desc;
+    uint32_t a_z, a_tab, a_part, a_c16, a_desc, a_cm;
 };
 
 // ---------------------------------------------------------------------------
@@ -112,6 +115,15 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+// Shared load at a 32-bit shared address plus a constant byte offset.  Not
+// volatile, so the compiler may schedule it; its address always derives from a
+// descriptor loaded after the barrier that publishes the tables.
+template <int OFF>
+__device__ __forceinline__ float lds_f32_imm(uint32_t addr) {
+    float v;
+    asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
     return v;
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -199,27 +211,60 @@ __device__ __forceinline__ void decode_pw(const UnitInfo& U, int q, int& g, int&
     w = rel - jb * W;
 }
 
+// Tasks [t0, t1) of a CTA.  With no more units than CTAs, every CTA works on
+// one unit only (units get floor or ceil of G/U CTAs, each a contiguous range
+// of the unit's row blocks), so each CTA builds one unit's tables; otherwise
+// the task list is cut into G contiguous pieces.
+__host__ __device__ inline void cta_tasks(const T1Params& P, int cta, int& t0, int& t1) {
+    const int U = 2 * P.K;
+    if (U <= P.G) {
+        const int u = (int)(((long long)cta * U) / P.G);
+        const int c0 = (int)(((long long)u * P.G + U - 1) / U), c1 = (int)(((long long)(u + 1) * P.G + U - 1) / U);
+        const int n = c1 - c0, i = cta - c0;
+        t0 = u * P.n_rb + (int)(((long long)i * P.n_rb) / n);
+        t1 = u * P.n_rb + (int)(((long long)(i + 1) * P.n_rb) / n);
+    } else {
+        t0 = (int)(((long long)cta * P.n_tasks) / P.G);
+        t1 = (int)(((long long)(cta + 1) * P.n_tasks) / P.G);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+// A run is a maximal set of consecutive tasks of this CTA that share a unit;
+// its staged plane words are laid out [plane word][rows of the run].
+struct RunInfo {
+    int ui;        // unit index inside the CTA
+    int t_first;   // first task
+    int nt;        // tasks in the run
+    int rows;      // staged rows (nt * kRB, clamped to d_pad)
+    uint32_t off;  // word offset of the run in the staging buffer
+};
+constexpr int kMaxRuns = kMaxUnitsPerCta;
+constexpr int kRunTasks = 4;  // tasks evaluated together (one accumulator each)
+
 __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t s_bar[kPhiBars];
+    __shared__ uint64_t s_bar[kPhiBars + 1];  // Phi chunks, then planes + metadata
     __shared__ UnitInfo s_unit[kMaxUnitsPerCta];
-    __shared__ int s_abort;
+    __shared__ RunInfo s_run[kMaxRuns];
+    __shared__ int s_abort, s_nruns;
     __shared__ unsigned long long s_bar_base;
     __shared__ float s_zp;
     __shared__ float s_zpw[kT1Warps];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cta = blockIdx.x;
-    const int t0 = (int)(((long long)cta * P.n_tasks) / P.G);
-    const int t1 = (int)(((long long)(cta + 1) * P.n_tasks) / P.G);
+    int t0, t1;
+    cta_tasks(P, cta, t0, t1);
     const int u_first = t0 / P.n_rb;
     const int u_last = t1 > t0 ? (t1 - 1) / P.n_rb : u_first - 1;
+    const int nunits = u_last - u_first + 1;
     const int rows_total = 2 * P.r;
     const int row0 = (int)(((long long)cta * rows_total) / P.G);
     const int row1 = (int)(((long long)(cta + 1) * rows_total) / P.G);
+    const int nrows = row1 - row0;
     const uint32_t row_bytes = (uint32_t)P.d_in * 2;
 
     uint16_t* s_x = reinterpret_cast<uint16_t*>(smem + P.sm_x);
@@ -227,20 +272,18 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
     uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);
     uint8_t* s_meta = smem + P.sm_meta;
 
-    // ---- phase 0: issue every HBM read: Phi rows and x first (they need nothing) ----
+    // ---- phase 0: Phi rows and x first (they need nothing), by one thread ----
     if (tid == 0) {
-        for (int i = 0; i < kPhiBars; i++) mbar_init(&s_bar[i], 1);
+        for (int i = 0; i <= kPhiBars; i++) mbar_init(&s_bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
         s_bar_base = ld_relaxed_u64(P.barrier);
-        const int nrows = row1 - row0;
         for (int bi = 0; bi < kPhiBars; bi++) {
             const int ra = row0 + (nrows * bi) / kPhiBars, rbnd = row0 + (nrows * (bi + 1)) / kPhiBars;
             uint32_t bytes = (uint32_t)(rbnd - ra) * row_bytes + (bi == 0 ? row_bytes : 0);
             mbar_expect_tx(&s_bar[bi], bytes);
             if (bi == 0) bulk_g2s(s_x, P.x, row_bytes, &s_bar[0]);
-            // rows [ra, rbnd) are contiguous inside each projection: at most two copies
-            for (int rr = ra; rr < rbnd;) {
+            for (int rr = ra; rr < rbnd;) {  // rows are contiguous inside a projection
                 const int p = rr / P.r, k = rr - p * P.r;
                 const int n = min(rbnd - rr, P.r - k);
                 bulk_g2s(s_a + (size_t)(rr - row0) * row_bytes, P.proj[p].phi_t + (size_t)k * P.d_in,
@@ -250,49 +293,82 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
         }
     }
     // routed experts of this CTA's units (two dependent reads: ids, then the directory)
-    if (tid >= 32 && tid - 32 < u_last - u_first + 1) unit_info(P, u_first + tid - 32, s_unit[tid - 32]);
-    __syncthreads();
+    if (warp == 1 && lane < nunits) unit_info(P, u_first + lane, s_unit[lane]);
+    __syncthreads();  // s_unit ready
 
-    // bit planes of this CTA's tasks: 32 rows x 4 B per plane word, 16 B per cp.async
-    const int nunits = u_last - u_first + 1;
-    for (int t = t0; t < t1; t++) {
-        const UnitInfo& U = s_unit[t / P.n_rb - u_first];
-        if (U.e < 0) continue;
-        const int rb = t % P.n_rb;
-        const uint8_t* blob = P.proj[U.p].blob;
-        uint32_t* dst = s_planes + (size_t)(t - t0) * P.pw_max * kRB;
-        for (int c = tid; c < U.pw * (kRB / 4); c += kT1Threads) {
-            const int q = c / (kRB / 4), chunk = c % (kRB / 4);
-            int g, jb, w;
-            decode_pw(U, q, g, jb, w);
-            const int row = rb * kRB + chunk * 4;
-            const int W = (int)(U.np[g] / 32);
-            const uint8_t* src = blob + U.planes_off[g] + 4 * (((uint64_t)jb * W + w) * P.d_pad + (uint64_t)row);
-            const bool ok = row < P.d_pad;  // d_pad % 8 == 0: a 4-row chunk is all in or all out
-            cp_async16(dst + (size_t)q * kRB + chunk * 4, ok ? src : blob, ok ? 16u : 0u);
+    // runs of this CTA's tasks (one thread)
+    if (tid == 32) {
+        int nr = 0;
+        uint32_t off = 0;
+        for (int t = t0; t < t1;) {
+            const int ui = t / P.n_rb - u_first;
+            const int te = min(t1, (ui + u_first + 1) * P.n_rb);
+            while (t < te) {
+                const int nt = min(kRunTasks, te - t);
+                RunInfo R;
+                R.ui = ui;
+                R.t_first = t;
+                R.nt = nt;
+                R.rows = nt * kRB;
+                R.off = off;
+                const UnitInfo& U = s_unit[ui];
+                off += (uint32_t)(U.e >= 0 ? U.pw : 0) * (uint32_t)(nt * kRB);
+                s_run[nr++] = R;
+                t += nt;
+            }
+        }
+        s_nruns = nr;
+        // bit planes (one copy per run, tile and group: the group's b x W x 32 words of a
+        // 32-row tile are contiguous) and per-component metadata (one copy per group)
+        uint32_t bytes = 0;
+        for (int ri = 0; ri < nr; ri++) {
+            const UnitInfo& U = s_unit[s_run[ri].ui];
+            if (U.e >= 0) bytes += 128u * (uint32_t)U.pw * (uint32_t)s_run[ri].nt;
+        }
+        for (int ui = 0; ui < nunits; ui++) {
+            const UnitInfo& U = s_unit[ui];
+            if (U.e < 0) continue;
+            for (int g = 0; g < kNumGroups; g++) bytes += (group_width(g) == 16 ? 6u : 8u) * U.np[g];
+        }
+        mbar_expect_tx(&s_bar[kPhiBars], bytes);
+        for (int ri = 0; ri < nr; ri++) {
+            const RunInfo& R = s_run[ri];
+            const UnitInfo& U = s_unit[R.ui];
+            if (U.e < 0) continue;
+            const uint8_t* blob = P.proj[U.p].blob;
+            const int tile0 = R.t_first % P.n_rb;
+            for (int k = 0; k < R.nt; k++)
+                for (int g = 1; g < kNumGroups; g++) {
+                    if (U.n[g] == 0) continue;
+                    const uint32_t gw = (uint32_t)group_width(g) * (U.np[g] / 32) * kRB;  // words per tile
+                    bulk_g2s(s_planes + R.off + (size_t)k * U.pw * kRB + (size_t)U.pw0[g] * kRB,
+                             blob + U.planes_off[g] + 4ull * gw * (uint64_t)(tile0 + k), 4u * gw, &s_bar[kPhiBars]);
+                }
+        }
+        for (int ui = 0; ui < nunits; ui++) {
+            const UnitInfo& U = s_unit[ui];
+            if (U.e < 0) continue;
+            const uint8_t* blob = P.proj[U.p].blob;
+            const DirEntry d = read_dir(blob, U.e);
+            for (int g = 0; g < kNumGroups; g++) {
+                if (U.n[g] == 0) continue;
+                bulk_g2s(s_meta + (size_t)ui * P.meta_max + U.meta_off[g], blob + d.base + d.goff[g],
+                         (group_width(g) == 16 ? 6u : 8u) * U.np[g], &s_bar[kPhiBars]);
+            }
         }
     }
-    // per-component metadata (idx, scale, amp) of this CTA's units
-    for (int ui = 0; ui < nunits; ui++) {
-        const UnitInfo& U = s_unit[ui];
-        if (U.e < 0) continue;
-        const uint8_t* blob = P.proj[U.p].blob;
-        const DirEntry d = read_dir(blob, U.e);
-        for (int g = 0; g < kNumGroups; g++) {
-            if (U.n[g] == 0) continue;
-            const uint32_t bytes = (group_width(g) == 16 ? 6u : 8u) * U.np[g];
-            const uint8_t* src = blob + d.base + d.goff[g];
-            uint8_t* dst = s_meta + (size_t)ui * P.meta_max + U.meta_off[g];
-            for (uint32_t o = (uint32_t)tid * 16; o < bytes; o += kT1Threads * 16) cp_async16(dst + o, src + o, 16);
-        }
-    }
-    cp_async_commit();
 
-    // ---- phase 1: z rows of this CTA ----
-    {
-        const int nrows = row1 - row0;
+    // ---- phase 1: z rows of this CTA on every warp but warp 1 (which issues the plane copies) ----
+    // The grid barrier is split: thread 0 arrives as soon as the row warps are
+    // done (named barrier 1), and waits only after that.  The counter is a
+    // multiple of G whenever no launch is in flight (it starts at zero and every
+    // launch adds exactly G), so the value read at start rounded down to a
+    // multiple of G is this launch's base.
+    if (warp != 1) {
+        const int wv = warp == 0 ? kT1Warps - 2 : warp - 2;  // 0 .. kT1Warps-2
+        constexpr int kRowWarps = kT1Warps - 1;
         bool ok = nrows == 0 || mbar_wait(&s_bar[0], 0);  // barrier 0 carries x
-        for (int rl = warp; ok && rl < nrows; rl += kT1Warps) {
+        for (int rl = wv; ok && rl < nrows; rl += kRowWarps) {
             int bi = 0;
             while (bi + 1 < kPhiBars && rl >= (nrows * (bi + 1)) / kPhiBars) bi++;
             if (!mbar_wait(&s_bar[bi], 0)) {
@@ -321,21 +397,20 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
             }
         }
         if (!ok) s_abort = 1;
-        // every bulk copy into this CTA's shared memory must have landed before it can exit
-        if (tid == 0)
+        asm volatile("bar.sync 1, %0;" ::"n"(kRowWarps * 32) : "memory");
+        if (tid == 0) {
+            // every bulk copy of Phi into this CTA's shared memory has landed (bounded)
             for (int bi = 0; bi < kPhiBars; bi++)
                 if (!mbar_wait(&s_bar[bi], 0)) s_abort = 1;
+            red_add_release_u64(P.barrier, 1ull);  // arrive
+        }
     }
-    __syncthreads();
+    __syncthreads();  // warp 1 has issued its copies; s_run is visible
 
-    // ---- grid barrier (bounded) ----
-    // The counter is a multiple of G whenever no launch is in flight (it starts
-    // at zero and every launch adds exactly G), so the value read at start
-    // rounded down to a multiple of G is this launch's base.
+    // ---- grid barrier wait (bounded), then the planes ----
     if (tid == 0) {
         const unsigned long long G = (unsigned long long)P.G;
         const unsigned long long target = (s_bar_base / G + 1) * G;
-        red_add_release_u64(P.barrier, 1ull);
         if (ld_acquire_u64(P.barrier) < target) {
             const long long tw = globaltimer();
             while (ld_acquire_u64(P.barrier) < target) {
@@ -345,82 +420,89 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
                 }
             }
         }
+        if (!mbar_wait(&s_bar[kPhiBars], 0)) s_abort = 1;  // planes and metadata
         if (s_abort && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
     }
     __syncthreads();
-    if (s_abort) {
-        cp_async_wait_all();
-        return;
-    }
+    if (s_abort) return;
 
-    // ---- phase 2: z of both projections into shared memory, then tasks ----
+    // ---- phase 2: z of the needed projections, then the runs ----
     float* s_z = reinterpret_cast<float*>(s_a + P.a_z);
-    // tables must start on a 64-byte shared-memory boundary (lookups OR the entry offset into the base)
-    float* s_tab = reinterpret_cast<float*>(s_a + P.a_tab + ((64u - (smem_u32(s_a + P.a_tab) & 63u)) & 63u));
+    // tables start on a 512-byte shared-memory boundary: one word's 8 tables are 512 B, so the
+    // byte address of a word's tables has a zero low byte and a lookup can splice the entry
+    // offset into it with one byte permute
+    float* s_tab = reinterpret_cast<float*>(s_a + P.a_tab + ((512u - (smem_u32(s_a + P.a_tab) & 511u)) & 511u));
     float* s_part = reinterpret_cast<float*>(s_a + P.a_part);
     float* s_c16 = reinterpret_cast<float*>(s_a + P.a_c16);
-    for (int i = tid; i < 2 * P.r; i += kT1Threads) s_z[i] = __ldcg(P.zbuf + i);
-    cp_async_wait_all();
-    __syncthreads();
-
     uint2* s_desc = reinterpret_cast<uint2*>(s_a + P.a_desc);
+    float* s_cm = reinterpret_cast<float*>(s_a + P.a_cm);
     const uint32_t tab_sbase = smem_u32(s_tab);
+    {
+        bool need[2] = {false, false};
+        for (int ui = 0; ui < nunits; ui++) need[s_unit[ui].p] = true;
+        for (int p = 0; p < 2; p++)
+            if (need[p])
+                for (int i = tid; i < P.r; i += kT1Threads) s_z[p * P.r + i] = __ldcg(P.zbuf + p * P.r + i);
+    }
+    __syncthreads();
     int cur_unit = -1;
-    for (int t = t0; t < t1; t++) {
-        const int ui = t / P.n_rb - u_first;
-        const UnitInfo& U = s_unit[ui];
-        const int rb = t % P.n_rb;
-        const int row = rb * kRB + lane;
-        if (ui != cur_unit && U.e >= 0) {
+    const int nruns = s_nruns;
+    for (int ri = 0; ri < nruns; ri++) {
+        const RunInfo R = s_run[ri];
+        const UnitInfo& U = s_unit[R.ui];
+        if (R.ui != cur_unit && U.e >= 0) {
             __syncthreads();  // the previous unit's tables and descriptors are no longer read
-            // nibble tables and the zero-point term of this unit
-            const uint8_t* meta = s_meta + (size_t)ui * P.meta_max;
+            const uint8_t* meta = s_meta + (size_t)R.ui * P.meta_max;
             const float* z = s_z + U.p * P.r;
             float zp = 0.0f;
-            for (int tb = tid; tb < U.ntab; tb += kT1Threads) {
-                int g = 1;
-#pragma unroll
-                for (int gg = 2; gg < kNumGroups; gg++)
-                    if ((uint32_t)tb >= U.tab0[gg]) g = gg;
-                const uint32_t np = U.np[g];
+            // pass 1: c_k = a_k s_k z_k of every member (bit-plane groups, concatenated in
+            // group order and padded: member m of table tb is 4 tb + (m % 4)), and the
+            // zero-point partial sums.  Group fields are copied to registers first: the
+            // stores below go to shared memory, where UnitInfo also lives.
+            for (int g = 1; g < kNumGroups; g++) {
+                const uint32_t np = U.np[g], n = U.n[g], m0 = 4 * U.tab0[g];
+                if (np == 0) continue;
                 const uint8_t* gm = meta + U.meta_off[g];
-                const uint16_t* idx = reinterpret_cast<const uint16_t*>(gm);
-                const uint16_t* scl = reinterpret_cast<const uint16_t*>(gm + 2 * np);
-                const float* amp = reinterpret_cast<const float*>(gm + 4 * np);
-                const uint32_t m0 = 4 * (tb - U.tab0[g]);
-                float c[4];
-#pragma unroll
-                for (int b = 0; b < 4; b++) {
-                    const uint32_t m = m0 + b;
-                    c[b] = m < U.n[g] ? amp[m] * __half2float(__ushort_as_half(scl[m])) * z[idx[m]] : 0.0f;
+                const float* __restrict__ amp = reinterpret_cast<const float*>(gm + 4 * np);
+                const uint16_t* __restrict__ scl = reinterpret_cast<const uint16_t*>(gm + 2 * np);
+                const uint16_t* __restrict__ idx = reinterpret_cast<const uint16_t*>(gm);
+                const float hr = 0.5f * (float)((1 << group_width(g)) - 1);
+                for (uint32_t ml = tid; ml < np; ml += kT1Threads) {
+                    float c = 0.0f;
+                    if (ml < n) c = amp[ml] * __half2float(__ushort_as_half(scl[ml])) * z[idx[ml]];
+                    s_cm[m0 + ml] = c;
+                    zp += hr * c;
                 }
-                float e[16];
-                e[0] = 0.0f;
-                e[1] = c[0];
-                e[2] = c[1];
-                e[3] = c[0] + c[1];
+            }
+            __syncthreads();
+            // pass 2: entry n of table tb = sum of c over the set bits of n (one entry per
+            // thread and step; four steps' loads are issued before their stores)
+            {
+                const int nent = 16 * U.ntab;
+                const float4* __restrict__ cm4 = reinterpret_cast<const float4*>(s_cm);
+                float* __restrict__ tab = s_tab;
+                const int n = tid & 15;  // kT1Threads is a multiple of 16: n is fixed per thread
+                for (int en0 = tid; en0 < nent; en0 += 4 * kT1Threads) {
+                    float4 c4[4];
 #pragma unroll
-                for (int h = 0; h < 4; h++) e[4 + h] = e[h] + c[2];
+                    for (int u = 0; u < 4; u++) {
+                        const int en = en0 + u * kT1Threads;
+                        c4[u] = en < nent ? cm4[en >> 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
 #pragma unroll
-                for (int h = 0; h < 8; h++) e[8 + h] = e[h] + c[3];
-                float4* dst = reinterpret_cast<float4*>(s_tab + 16 * tb);
-                dst[0] = make_float4(e[0], e[1], e[2], e[3]);
-                dst[1] = make_float4(e[4], e[5], e[6], e[7]);
-                dst[2] = make_float4(e[8], e[9], e[10], e[11]);
-                dst[3] = make_float4(e[12], e[13], e[14], e[15]);
-                zp += 0.5f * (float)((1 << group_width(g)) - 1) * ((c[0] + c[1]) + (c[2] + c[3]));
+                    for (int u = 0; u < 4; u++) {
+                        const int en = en0 + u * kT1Threads;
+                        if (en < nent)
+                            tab[en] = ((n & 1 ? c4[u].x : 0.0f) + (n & 2 ? c4[u].y : 0.0f)) +
+                                      ((n & 4 ? c4[u].z : 0.0f) + (n & 8 ? c4[u].w : 0.0f));
+                    }
+                }
             }
             // plane-word descriptors: shared-memory byte offset of the word's 8 tables, weight 2^j
             for (int q = tid; q < U.pw; q += kT1Threads) {
-                int g = 1;
-#pragma unroll
-                for (int gg = 2; gg < kNumGroups; gg++)
-                    if ((uint32_t)q >= U.pw0[gg]) g = gg;
-                const int W = (int)(U.np[g] / 32);
-                const int rel = q - (int)U.pw0[g];
-                const int jb = rel / W, w = rel - jb * W;
-                s_desc[q] = make_uint2(tab_sbase + 64u * (U.tab0[g] + 8u * (uint32_t)w),
-                                       __float_as_uint((float)(1u << jb)));
+                int g, jb, w;
+                decode_pw(U, q, g, jb, w);
+                s_desc[q] = make_uint2(tab_sbase + 64u * (U.tab0[g] + 8u * (uint32_t)w), __float_as_uint((float)(1u << jb)));
             }
             if (U.n16 > 0) {
                 const uint8_t* gm = meta + U.meta_off[0];
@@ -431,43 +513,66 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
             zp = warp_sum(zp);
             if (lane == 0) s_zpw[warp] = zp;
             __syncthreads();
-            if (tid == 0) {
-                float sum = 0.0f;
-                for (int w = 0; w < kT1Warps; w++) sum += s_zpw[w];
-                s_zp = sum;
+            if (warp == 0) {
+                float v = lane < kT1Warps ? s_zpw[lane] : 0.0f;
+                v = warp_sum(v);
+                if (lane == 0) s_zp = v;
             }
             __syncthreads();
-            cur_unit = ui;
+            cur_unit = R.ui;
         }
-        float acc = 0.0f;
+        // every warp takes a share of the unit's plane words for all tasks of the run
+        float acc[kRunTasks];
+#pragma unroll
+        for (int k = 0; k < kRunTasks; k++) acc[k] = 0.0f;
         if (U.e >= 0) {
-            const uint32_t* pl = s_planes + (size_t)(t - t0) * P.pw_max * kRB + lane;
+            const int stride = U.pw * kRB;  // words between consecutive tasks (tiles) of the run
+            const uint32_t* pl = s_planes + R.off + lane;
             for (int q = warp; q < U.pw; q += kT1Warps) {
                 const uint2 d = s_desc[q];
-                const uint32_t word = pl[q * kRB];
-                // table t of this word sits at d.x + 64 t (64-byte aligned), entry n at + 4 n
-                float l[8];
+                const float wt = __uint_as_float(d.y);
 #pragma unroll
-                for (int n = 0; n < 8; n++) {
-                    const uint32_t off = n == 0 ? ((word << 2) & 0x3Cu) : ((word >> (4 * n - 2)) & 0x3Cu);
-                    l[n] = lds_f32((d.x | off) + 64u * n);
+                for (int k = 0; k < kRunTasks; k++) {
+                    if (k < R.nt) {
+                        const uint32_t word = pl[k * stride + q * kRB];
+                        // entry offsets (nibble x 4 bytes): even nibbles in the bytes of lo, odd in hi;
+                        // table n of this word is at d.x + 64 n, entry e at + 4 e
+                        const uint32_t lo = (word << 2) & 0x3C3C3C3Cu, hi = (word >> 2) & 0x3C3C3C3Cu;
+                        float l[8];
+                        l[0] = lds_f32_imm<0>(__byte_perm(lo, d.x, 0x7650u));
+                        l[1] = lds_f32_imm<64>(__byte_perm(hi, d.x, 0x7650u));
+                        l[2] = lds_f32_imm<128>(__byte_perm(lo, d.x, 0x7651u));
+                        l[3] = lds_f32_imm<192>(__byte_perm(hi, d.x, 0x7651u));
+                        l[4] = lds_f32_imm<256>(__byte_perm(lo, d.x, 0x7652u));
+                        l[5] = lds_f32_imm<320>(__byte_perm(hi, d.x, 0x7652u));
+                        l[6] = lds_f32_imm<384>(__byte_perm(lo, d.x, 0x7653u));
+                        l[7] = lds_f32_imm<448>(__byte_perm(hi, d.x, 0x7653u));
+                        const float sum = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
+                        acc[k] = fmaf(sum, wt, acc[k]);
+                    }
                 }
-                const float sum = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
-                acc = fmaf(sum, __uint_as_float(d.y), acc);
             }
-            if (U.n16 > 0 && row < P.d_out) {
+            if (U.n16 > 0) {
                 const uint16_t* w16 = reinterpret_cast<const uint16_t*>(P.proj[U.p].blob + U.w16_off);
-                for (int m = warp; m < U.n16; m += kT1Warps)
-                    acc = fmaf(s_c16[m], __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row])), acc);
+#pragma unroll
+                for (int k = 0; k < kRunTasks; k++) {
+                    const int row = ((R.t_first + k) % P.n_rb) * kRB + lane;
+                    if (k < R.nt && row < P.d_out)
+                        for (int m = warp; m < U.n16; m += kT1Warps)
+                            acc[k] = fmaf(s_c16[m], __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row])),
+                                          acc[k]);
+                }
             }
         }
-        s_part[warp * kRB + lane] = acc;
+#pragma unroll
+        for (int k = 0; k < kRunTasks; k++) s_part[(k * kT1Warps + warp) * kRB + lane] = acc[k];
         __syncthreads();
-        if (warp == 0) {
+        if (warp < R.nt) {  // warp k reduces task k of the run
+            const int k = warp, t = R.t_first + k, rb = t % P.n_rb, row = rb * kRB + lane;
             float y = 0.0f;
             if (U.e >= 0) {
 #pragma unroll
-                for (int w = 0; w < kT1Warps; w++) y += s_part[w * kRB + lane];
+                for (int w = 0; w < kT1Warps; w++) y += s_part[(k * kT1Warps + w) * kRB + lane];
                 y -= s_zp;
             }
             if (row < P.d_out) {
@@ -572,7 +677,14 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     P.n_rb = (P.d_out + kRB - 1) / kRB;
     P.n_tasks = 2 * P.K * P.n_rb;
     P.phi_rows = (2 * P.r + P.G - 1) / P.G;
-    P.tasks_max = (P.n_tasks + P.G - 1) / P.G;
+    P.tasks_max = 0;
+    int units_max = 0;
+    for (int c = 0; c < P.G; c++) {  // exact bounds of the partition the kernel uses
+        int a, b;
+        cta_tasks(P, c, a, b);
+        P.tasks_max = std::max(P.tasks_max, b - a);
+        if (b > a) units_max = std::max(units_max, (b - 1) / P.n_rb - a / P.n_rb + 1);
+    }
     int pw = 0, members = 0, meta = 0, n16 = 0;
     unit_bounds(g, pw, members, meta, n16);
     unit_bounds(u, pw, members, meta, n16);
@@ -580,16 +692,18 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     P.members_max = members;
     P.meta_max = align_up(meta, 16);
     P.n16_max = n16;
-    const int units_max = (P.tasks_max + P.n_rb - 1) / P.n_rb + 1;
+
     if (units_max > kMaxUnitsPerCta || P.tasks_max > 64 || P.d_in % 8 || P.d_in > 8192) return L;
+    if (units_max + (P.tasks_max + kRunTasks - 1) / kRunTasks > kMaxRuns) return L;
     // shared memory
     const uint64_t phi_bytes = (uint64_t)P.phi_rows * P.d_in * 2;
     P.a_z = 0;
     P.a_tab = align_up(P.a_z + 8ull * P.r, 128);
-    P.a_part = align_up(P.a_tab + 64 + 16ull * 4 * (members / 4), 16);  // + 64: tables realigned in the kernel
-    P.a_c16 = align_up(P.a_part + 4ull * kT1Warps * kRB, 16);
+    P.a_part = align_up(P.a_tab + 512 + 16ull * 4 * (members / 4), 16);  // + 512: tables realigned in the kernel
+    P.a_c16 = align_up(P.a_part + 4ull * kRunTasks * kT1Warps * kRB, 16);
     P.a_desc = align_up(P.a_c16 + 4ull * n16, 16);
-    const uint64_t a_bytes = std::max<uint64_t>(phi_bytes, P.a_desc + 8ull * P.pw_max);
+    P.a_cm = align_up(P.a_desc + 8ull * P.pw_max, 16);
+    const uint64_t a_bytes = std::max<uint64_t>(phi_bytes, P.a_cm + 4ull * members);
     P.sm_x = 0;
     P.sm_a = align_up(P.sm_x + 2ull * P.d_in, 128);
     P.sm_planes = align_up(P.sm_a + a_bytes, 128);

@@ -114,7 +114,8 @@ static int orc_width_ok(int b) {
 
 static uint64_t orc_roundup(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
 
-/* Bytes of one group of width b holding n members, rows padded to d_pad. */
+/* Bytes of one group of width b holding n members, rows padded to d_pad
+ * (a multiple of 32: the planes are stored in 32-row tiles). */
 static uint64_t orc_group_bytes(int b, uint64_t n, uint64_t d_pad) {
     if (n == 0) return 0;
     if (b == 16) {
@@ -123,6 +124,12 @@ static uint64_t orc_group_bytes(int b, uint64_t n, uint64_t d_pad) {
     }
     uint64_t np = orc_roundup(n, 32);
     return 2 * np + 2 * np + 4 * np + 4 * (uint64_t)b * (np / 32) * d_pad; /* idx, scale, amp, planes */
+}
+
+/* Byte offset of plane word [tile i/32][plane j][word w][row i%32] inside a
+ * group's planes; W = words per plane. */
+static uint64_t orc_plane_off(uint64_t j, uint64_t w, uint64_t W, int b, uint64_t i) {
+    return 4 * ((((i / 32) * (uint64_t)b + j) * W + w) * 32 + i % 32);
 }
 
 /* Count of each width for expert e: cnt[g] for groups g = 0..6 (widths
@@ -149,7 +156,7 @@ static int orc_dims_ok(int E, int r, int d_out) {
 /* Total blob bytes for the given widths [E][r]; 0 on invalid input. */
 uint64_t orc_blob_bytes(int E, int r, int d_out, const uint8_t *widths) {
     if (!orc_dims_ok(E, r, d_out) || !widths) return 0;
-    uint64_t d_pad = orc_roundup((uint64_t)d_out, 8);
+    uint64_t d_pad = orc_roundup((uint64_t)d_out, 32);
     uint64_t total = 64 + 64 * (uint64_t)E;
     for (int e = 0; e < E; e++) {
         uint32_t cnt[8];
@@ -261,7 +268,7 @@ int orc_pack(int E, int r, int d_out, const uint8_t *widths, const float *comps,
     if (need == 0) return ORC_EWIDTH;
     if (blob_bytes < need) return ORC_ESIZE;
     memset(blob, 0, need);
-    uint64_t d_pad = orc_roundup((uint64_t)d_out, 8);
+    uint64_t d_pad = orc_roundup((uint64_t)d_out, 32);
     int32_t st = 0;
 
     /* header */
@@ -330,7 +337,7 @@ int orc_pack(int E, int r, int d_out, const uint8_t *widths, const float *comps,
                             uint32_t q = orc_quantise(p[i], b, sh, &st);
                             for (int j = 0; j < b; j++) {
                                 if (!((q >> j) & 1u)) continue;
-                                uint8_t *word = planes + 4 * (((uint64_t)j * W + w) * d_pad + (uint64_t)i);
+                                uint8_t *word = planes + orc_plane_off((uint64_t)j, w, W, b, (uint64_t)i);
                                 put32(word, get32(word) | (1u << bit));
                             }
                         }
@@ -359,7 +366,7 @@ int orc_blob_parse(const uint8_t *blob, uint64_t bytes, int *E, int *r, int *d_o
     if (!blob || bytes < 64) return ORC_EFORMAT;
     if (get32(blob) != 0x454F4D42u || get32(blob + 4) != 1u) return ORC_EFORMAT;
     uint64_t dout = get32(blob + 8), dpad = get32(blob + 12), ne = get32(blob + 16), rk = get32(blob + 20);
-    if (!orc_dims_ok((int)ne, (int)rk, (int)dout) || dpad != orc_roundup(dout, 8)) return ORC_EFORMAT;
+    if (!orc_dims_ok((int)ne, (int)rk, (int)dout) || dpad != orc_roundup(dout, 32)) return ORC_EFORMAT;
     uint64_t total = get64(blob + 24);
     if (total != bytes || get64(blob + 32) != 64u || get64(blob + 40) != 64u + 64u * ne) return ORC_EFORMAT;
     for (int i = 48; i < 64; i++)
@@ -398,7 +405,7 @@ int orc_unpack(const uint8_t *blob, uint64_t bytes, uint16_t *q, uint8_t *widths
     int E, r, d_out;
     int rc = orc_blob_parse(blob, bytes, &E, &r, &d_out);
     if (rc) return rc;
-    uint64_t d_pad = orc_roundup((uint64_t)d_out, 8);
+    uint64_t d_pad = orc_roundup((uint64_t)d_out, 32);
     if (q) memset(q, 0, sizeof(uint16_t) * (size_t)E * r * d_out);
     if (widths) memset(widths, 0, (size_t)E * r);
     if (scales) memset(scales, 0, sizeof(uint16_t) * (size_t)E * r);
@@ -443,7 +450,7 @@ int orc_unpack(const uint8_t *blob, uint64_t bytes, uint16_t *q, uint8_t *widths
                         for (int i = 0; i < d_out; i++) {
                             uint32_t v = 0;
                             for (int j = 0; j < b; j++) {
-                                uint32_t word = get32(planes + 4 * (((uint64_t)j * W + m / 32) * d_pad + (uint64_t)i));
+                                uint32_t word = get32(planes + orc_plane_off((uint64_t)j, m / 32, W, b, (uint64_t)i));
                                 v |= ((word >> (m % 32)) & 1u) << j;
                             }
                             q[ek * d_out + i] = (uint16_t)v;
@@ -521,7 +528,7 @@ int orc_expert_forward(const uint8_t *blob, uint64_t bytes, const double *Z, con
     int rc = orc_blob_parse(blob, bytes, &E, &r, &d_out);
     if (rc) return rc;
     if (T < 0 || top_k < 1 || !Z || !ids || !g || !Y_sum) return ORC_EINVAL;
-    uint64_t d_pad = orc_roundup((uint64_t)d_out, 8);
+    uint64_t d_pad = orc_roundup((uint64_t)d_out, 32);
     int32_t st = 0;
     double *y = (double *)malloc(sizeof(double) * (size_t)d_out);
     if (!y) return ORC_EINVAL;
@@ -557,7 +564,7 @@ int orc_expert_forward(const uint8_t *blob, uint64_t bytes, const double *Z, con
                                 uint64_t W = np / 32;
                                 uint32_t v = 0;
                                 for (int j = 0; j < b; j++) {
-                                    uint32_t word = get32(G + 8 * np + 4 * (((uint64_t)j * W + m / 32) * d_pad + (uint64_t)i));
+                                    uint32_t word = get32(G + 8 * np + orc_plane_off((uint64_t)j, m / 32, W, b, (uint64_t)i));
                                     v |= ((word >> (m % 32)) & 1u) << j;
                                 }
                                 qv = (uint16_t)v;
