@@ -153,6 +153,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 namespace bitsmoe {
 int set_cuda_error(cudaError_t e);  // records the text, returns BITSMOE_ECUDA
 int check_launch();                 // cudaGetLastError -> 0 or ECUDA
+
+// Routing groups of one call (in the caller's workspace).
+struct RouteWS {
+    int32_t* count;    // [E]   (reused as the scatter cursor)
+    int32_t* start;    // [E+1] first pair of each expert in `pairs`
+    int32_t* active;   // [E]   experts with at least one pair, ascending
+    int32_t* nactive;  // [1]
+    int32_t* pairs;    // [T*K] pair index t*K + j, grouped by expert
+};
 }  // namespace bitsmoe
 
 // The plan object (host).

@@ -20,13 +20,6 @@ int launch_shared_proj(const uint16_t* phi_t, const uint16_t* X, float* Z, int T
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------
-struct RouteWS {
-    int32_t* count;    // [E]   (reused as the scatter cursor)
-    int32_t* start;    // [E+1] first pair of each expert in `pairs`
-    int32_t* active;   // [E]   experts with at least one pair, ascending
-    int32_t* nactive;  // [1]
-    int32_t* pairs;    // [T*K] pair index t*K + j, grouped by expert
-};
 
 struct WsCursor {
     uint8_t* p;
@@ -108,136 +101,6 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(const int32_t* __restri
     }
 }
 
-// ---------------------------------------------------------------------------
-// expert forward, general form: one CTA per (active expert, row block)
-// ---------------------------------------------------------------------------
-constexpr int kExThreads = 256;
-constexpr int kTC = 4;       // tokens per pass
-constexpr int kMCH = 1024;   // members per c-table chunk (multiple of 32)
-
-__global__ void __launch_bounds__(kExThreads) k_expert_general(const uint8_t* __restrict__ blob,
-                                                               const float* __restrict__ Z, int r, int K, int d_out,
-                                                               uint32_t d_pad, RouteWS ws, float* __restrict__ Ye) {
-    __shared__ float s_c[kMCH][kTC];
-    __shared__ float s_zp[kExThreads / 32][kTC];
-    __shared__ int s_pair[kTC];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int slot = blockIdx.x;
-    if (slot >= *ws.nactive) return;
-    const int e = ws.active[slot];
-    const int p0 = ws.start[e], p1 = ws.start[e + 1];
-    const DirEntry d = read_dir(blob, e);
-    const uint32_t i = blockIdx.y * kExThreads + tid;  // this thread's row
-    const bool row_ok = i < (uint32_t)d_out;
-
-    for (int pc = p0; pc < p1; pc += kTC) {
-        const int nt = min(kTC, p1 - pc);
-        __syncthreads();
-        if (tid < kTC) s_pair[tid] = tid < nt ? ws.pairs[pc + tid] : -1;
-        __syncthreads();
-        int tok[kTC];
-#pragma unroll
-        for (int j = 0; j < kTC; j++) tok[j] = s_pair[j] >= 0 ? s_pair[j] / K : -1;
-        float acc[kTC];
-#pragma unroll
-        for (int j = 0; j < kTC; j++) acc[j] = 0.0f;
-
-        for (int g = 0; g < kNumGroups; g++) {
-            const int b = group_width(g);
-            const uint32_t n = d.count[g];
-            if (n == 0) continue;
-            const uint32_t np = (uint32_t)group_members_padded(b, n);
-            const uint16_t *idx, *scl = nullptr;
-            const float* amp;
-            const uint32_t* planes = nullptr;
-            const uint16_t* w16 = nullptr;
-            if (b == 16) {
-                HGroup h = hgroup(blob, d);
-                idx = h.idx;
-                amp = h.amp;
-                w16 = h.w16;
-            } else {
-                QGroup q = qgroup(blob, d, g);
-                idx = q.idx;
-                scl = q.scale;
-                amp = q.amp;
-                planes = q.planes;
-            }
-            for (uint32_t m0 = 0; m0 < np; m0 += kMCH) {
-                const uint32_t m1 = min(np, m0 + kMCH);
-                __syncthreads();
-                float zl[kTC];
-#pragma unroll
-                for (int j = 0; j < kTC; j++) zl[j] = 0.0f;
-                for (uint32_t m = m0 + tid; m < m1; m += kExThreads) {
-                    float cs = 0.0f;
-                    int k = 0;
-                    if (m < n) {
-                        k = idx[m];
-                        cs = amp[m];
-                        if (b != 16) cs = cs * __half2float(__ushort_as_half(scl[m]));
-                    }
-#pragma unroll
-                    for (int j = 0; j < kTC; j++) {
-                        float c = (m < n && tok[j] >= 0) ? cs * Z[(uint64_t)tok[j] * r + k] : 0.0f;
-                        s_c[m - m0][j] = c;
-                        zl[j] += c;
-                    }
-                }
-                if (b != 16) {
-#pragma unroll
-                    for (int j = 0; j < kTC; j++) {
-                        float v = warp_sum(zl[j]);
-                        if (lane == 0) s_zp[warp][j] = v;
-                    }
-                }
-                __syncthreads();
-                if (b != 16) {  // zero-point term: -(2^b - 1)/2 * sum_k c_k, shared by all rows
-                    const float half_range = 0.5f * (float)((1 << b) - 1);
-#pragma unroll
-                    for (int j = 0; j < kTC; j++) {
-                        float zs = 0.0f;
-                        for (int w = 0; w < kExThreads / 32; w++) zs += s_zp[w][j];
-                        acc[j] -= half_range * zs;
-                    }
-                }
-                if (!row_ok) continue;
-                if (b == 16) {
-                    for (uint32_t m = m0; m < min(m1, n); m++) {
-                        float wv = __half2float(__ushort_as_half(w16[(uint64_t)m * d_pad + i]));
-#pragma unroll
-                        for (int j = 0; j < kTC; j++) acc[j] = fmaf(s_c[m - m0][j], wv, acc[j]);
-                    }
-                } else {
-                    const uint32_t W = np / 32;
-                    for (uint32_t w = m0 / 32; w < m1 / 32; w++) {
-                        for (int pb = 0; pb < b; pb++) {
-                            uint32_t word = planes[plane_word(pb, w, W, b, i)];
-                            const float wt = (float)(1u << pb);
-                            float part[kTC];
-#pragma unroll
-                            for (int j = 0; j < kTC; j++) part[j] = 0.0f;
-                            while (word) {
-                                int mm = __ffs(word) - 1;
-                                word &= word - 1;
-#pragma unroll
-                                for (int j = 0; j < kTC; j++) part[j] += s_c[32 * w + mm - m0][j];
-                            }
-#pragma unroll
-                            for (int j = 0; j < kTC; j++) acc[j] = fmaf(wt, part[j], acc[j]);
-                        }
-                    }
-                }
-            }
-        }
-        if (row_ok) {
-#pragma unroll
-            for (int j = 0; j < kTC; j++)
-                if (j < nt) Ye[(uint64_t)s_pair[j] * d_out + i] = acc[j];
-        }
-    }
-}
-
 // Y_sum[t][i] = sum_j g[t][j] Y_e[t][j][i]; rows of out-of-range ids are zeroed.
 __global__ void k_combine(const int32_t* __restrict__ ids, const float* __restrict__ gw, float* Ye,
                           float* __restrict__ Ysum, int T, int K, int E, int d_out) {
@@ -258,13 +121,14 @@ __global__ void k_combine(const int32_t* __restrict__ ids, const float* __restri
     }
 }
 
+int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, int T, const RouteWS& rw, float* Ye,
+                     int32_t* status, cudaStream_t s);
+
 static int launch_expert(const bitsmoe_plan* p, const void* blob, const float* Z, const int32_t* ids,
-                         const float* gw, int T, float* Ye, float* Ysum, const RouteWS& rw, cudaStream_t s) {
+                         const float* gw, int T, float* Ye, float* Ysum, const RouteWS& rw, int32_t* status,
+                         cudaStream_t s) {
     const int E = p->dims.n_experts, K = p->dims.top_k, d_out = p->dims.d_out;
-    const int slots = (int)std::min<int64_t>((int64_t)E, (int64_t)T * K);
-    dim3 grid((unsigned)slots, (unsigned)((d_out + kExThreads - 1) / kExThreads));
-    k_expert_general<<<grid, kExThreads, 0, s>>>((const uint8_t*)blob, Z, p->dims.rank, K, d_out, p->d_pad, rw, Ye);
-    int rc = check_launch();
+    int rc = launch_expert_mt(p, blob, Z, T, rw, Ye, status, s);
     if (rc) return rc;
     uint64_t n = (uint64_t)T * d_out;
     unsigned blocks = (unsigned)std::min<uint64_t>((n + 255) / 256, 4096);
@@ -312,7 +176,7 @@ BITSMOE_API int bitsmoe_expert_forward(const bitsmoe_plan* plan, const void* blo
     cudaStream_t s = (cudaStream_t)stream;
     int rc = launch_route(plan, topk_ids, T, rw, status, s);
     if (rc) return rc;
-    return launch_expert(plan, blob, Z, topk_ids, gate_w, T, Ye, Y_sum, rw, s);
+    return launch_expert(plan, blob, Z, topk_ids, gate_w, T, Ye, Y_sum, rw, status, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -394,7 +258,7 @@ BITSMOE_API int bitsmoe_layer_forward(const bitsmoe_proj_io* gate, const bitsmoe
         float* Ye = io[j]->Y_experts ? io[j]->Y_experts : L.Ye[j];
         rc = launch_shared_proj(io[j]->phi_t, X, Z, T, p->dims.d_in, p->dims.rank, s);
         if (rc) return rc;
-        rc = launch_expert(p, io[j]->blob, Z, topk_ids, gate_w, T, Ye, io[j]->Y_sum, L.route, s);
+        rc = launch_expert(p, io[j]->blob, Z, topk_ids, gate_w, T, Ye, io[j]->Y_sum, L.route, status, s);
         if (rc) return rc;
     }
     return BITSMOE_OK;

@@ -3,7 +3,8 @@
 // every expert selected for the token reuses it).
 //
 // Phi^T is [r][d_in] fp16 (row k = phi_k, K-major), X is [T][d_in] fp16.
-// One warp owns one row of Phi^T; the row is read from HBM once, kept in
+// Batches of 8 or more tokens go to the tensor-core kernel (proj_tc.cu) when
+// r is a multiple of 128 and d_in of 512.  Otherwise one warp owns one row of Phi^T; the row is read from HBM once, kept in
 // registers, and dotted with every token of the batch (fp32 accumulation of
 // exact fp16 x fp16 products).  This is an HBM stream over Phi.
 #include "common.cuh"
@@ -65,9 +66,15 @@ __global__ void __launch_bounds__(kSPWarps * 32) k_shared_proj(const uint16_t* _
     }
 }
 
+bool proj_tc_supported(int T, int d_in, int r);
+int launch_proj_tc(const uint16_t* phi_t, const uint16_t* X, float* Z, int T, int d_in, int r, int32_t* status,
+                   cudaStream_t s);
+
+// T >= 8 tokens on the tensor cores when the shapes allow it, else the GEMV.
 int launch_shared_proj(const uint16_t* phi_t, const uint16_t* X, float* Z, int T, int d_in, int r,
                        cudaStream_t s) {
     if (T == 0) return BITSMOE_OK;
+    if (proj_tc_supported(T, d_in, r)) return launch_proj_tc(phi_t, X, Z, T, d_in, r, nullptr, s);
     dim3 grid((unsigned)((r + kSPWarps - 1) / kSPWarps));
     k_shared_proj<<<grid, kSPWarps * 32, 0, s>>>(phi_t, X, Z, T, d_in, r);
     return check_launch();
