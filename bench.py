@@ -335,6 +335,13 @@ def workload_config(cfg, T, n_layers, wl_bytes, touched):
             "routing": cfg.routing}
 
 
+def weak_scaling_throughput(world: int, steps: int, tokens: int, ms_max: float):
+    """Whole-job tokens/s and seconds per step: every rank runs `steps` steps of
+    `tokens` tokens on its own replica; the job takes the slowest rank's time."""
+    sec = ms_max / 1e3
+    return world * steps * tokens / sec, sec / steps
+
+
 def run_ours(args, dist):
     import numpy as np
     import torch
@@ -383,11 +390,8 @@ def run_ours(args, dist):
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_pop()
     dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    ms = dist.max(ms)
-    sec = ms / 1e3
-    value = dist.world * K * T / sec
-    step_s = sec / K
+    ms = dist.max(ev0.elapsed_time(ev1))
+    value, step_s = weak_scaling_throughput(dist.world, K, T, ms)
 
     peak, peak_kind = load_peak()
     achieved = alg["total"] / step_s / 1e9
