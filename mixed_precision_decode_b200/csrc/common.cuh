@@ -66,8 +66,8 @@ struct DirEntry {
     uint32_t count[kNumGroups]; // members per group
 };
 
-__device__ inline DirEntry read_dir(const uint8_t* blob, int e) {
-    const uint8_t* d = blob + kHeaderBytes + kDirEntryBytes * (uint64_t)e;
+// Decodes the directory entry at d (global or shared memory).
+__device__ inline DirEntry parse_dir(const uint8_t* d) {
     DirEntry r;
     r.base = *reinterpret_cast<const uint64_t*>(d);
     const uint32_t* go = reinterpret_cast<const uint32_t*>(d + 16);
@@ -78,6 +78,10 @@ __device__ inline DirEntry read_dir(const uint8_t* blob, int e) {
         r.count[g] = ct[g];
     }
     return r;
+}
+
+__device__ inline DirEntry read_dir(const uint8_t* blob, int e) {
+    return parse_dir(blob + kHeaderBytes + kDirEntryBytes * (uint64_t)e);
 }
 
 // Pointers into one group of width b (1..8).

@@ -7,17 +7,25 @@
 // bit-serially:  y_i = sum_b sum_j 2^j sum_{k in G_b} c_k bit_{k,j,i}
 //                      - sum_b (2^b - 1)/2 sum_{k in G_b} c_k,  c_k = a_k s_k z_k.
 //
-// Design for B200 at one token: the step moves ~24 MB (Phi of both
+// Design for B200 at one token.  The step moves ~24 MB (Phi of both
 // projections dominates) and has one grid-wide dependency (every expert row
-// needs all of z).  So every CTA issues ALL of its HBM reads at launch --
-// its slice of Phi rows by TMA bulk copies into shared memory, its slice of
-// bit planes and per-component metadata by cp.async -- then computes its
-// z rows, meets the other CTAs at a bounded grid barrier, and evaluates its
-// (projection, slot, 32-row block) tasks from shared memory.  The bit-serial
-// sum over 32 members of one plane word uses eight 16-entry subset-sum tables
-// (one per nibble of members): one conflict-free shared-memory lookup per 4
-// bits.  The routed sum is done by the last CTA to finish each row block, in
-// slot order, so results do not depend on timing.
+// needs all of z).  Every CTA issues its HBM reads at launch -- its slice of
+// Phi rows by TMA bulk copies, its share of the routed bit planes and their
+// metadata by cp.async -- computes its z rows and meets the other CTAs at a
+// bounded grid barrier.
+//
+// The expert work is cut by COLUMNS: the routed units' plane words (one word
+// = one bit plane of 32 members, over all rows) and octets of fp16 members
+// are concatenated and every CTA takes an equal contiguous share of them, for
+// all rows.  So a CTA builds subset-sum tables only for the member words it
+// evaluates (no table is built twice except at share boundaries), and the
+// work per CTA differs by at most one word.  Warps own 32-row tiles; the sum
+// over 32 members of one plane word uses eight 16-entry tables (one per
+// nibble), one shared-memory lookup per 4 bits.  Each CTA adds its rows of
+// every unit it touched (with its share of the zero-point term subtracted) to
+// Y_e and, times the gate weight, to Y_sum with fp32 red.add, so the kernel
+// has one grid barrier; the order of those additions, and so the last bits
+// of the outputs, can differ from run to run.
 #include <algorithm>
 #include <mutex>
 
@@ -25,14 +33,14 @@
 
 namespace bitsmoe {
 
-#ifndef BITSMOE_T1_THREADS
-#define BITSMOE_T1_THREADS 512
-#endif
-constexpr int kT1Threads = BITSMOE_T1_THREADS;  // threads per CTA of the fused kernel
-constexpr int kT1Warps = kT1Threads / 32;
-constexpr int kRB = 32;            // rows per task (one per lane)
-constexpr int kMaxUnitsPerCta = 8;
-constexpr int kPhiBars = 4;        // mbarriers over the Phi slice
+constexpr int kT1MaxThreads = 768;
+constexpr int kT1MaxWarps = kT1MaxThreads / 32;
+constexpr int kRB = 32;           // rows per tile (one per lane)
+constexpr int kMaxUnits = 32;     // routed (projection, slot) pairs: 2 * top_k
+constexpr int kMaxItems = 32;     // work items per CTA (one planning lane each)
+constexpr int kF16Item = 8;       // fp16 members per item
+constexpr int kStageWarps = 1;    // warps that issue the plane and metadata copies
+constexpr int kPhiBars = 4;       // mbarriers over the Phi slice
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded waits: 2 s, then BITSMOE_ST_TIMEOUT
 
 struct T1Proj {
@@ -49,21 +57,13 @@ struct T1Params {
     const int32_t* ids;
     const float* gw;
     int32_t* status;
-    unsigned long long* barrier;  // persistent, zero-initialised once
-    uint32_t* rb_count;           // [2][n_rb], persistent, zero-initialised once
+    unsigned long long* barrier;  // persistent, zero-initialised once; G arrivals per launch
     float* zbuf;                  // [2][r]
-    float* scratch;               // [2][K][d_pad]: g_j * y for the ordered combine
-    int d_in, d_out, d_pad, r, K, E;
-    int n_rb, n_tasks, G;
-    int phi_rows;       // Phi rows per CTA (last CTA may have fewer)
-    int tasks_max;      // tasks per CTA (upper bound)
-    int pw_max;         // plane words per unit (upper bound over both blobs)
-    int members_max;    // padded bit-plane members per unit (upper bound)
-    int meta_max;       // metadata bytes per unit (upper bound)
-    int n16_max;        // fp16 members per unit (upper bound)
-    // shared-memory layout (byte offsets)
-    uint32_t sm_x, sm_a, sm_planes, sm_meta, sm_end;
-    uint32_t a_z, a_tab, a_part, a_c16, a_desc, a_cm;
+    int d_in, d_out, d_pad, r, K, E, U;
+    int n_rb, G;
+    int items_max;  // work items per CTA (upper bound over every routing)
+    // dynamic shared-memory layout (byte offsets)
+    uint32_t sm_x, sm_dir, sm_phi, sm_planes, sm_mw, sm_f16, sm_c16, sm_tab, sm_end;
 };
 
 // ---------------------------------------------------------------------------
@@ -101,33 +101,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if (globaltimer() - t0 > kWaitLimitNs) return false;
     return true;
 }
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
+// Bulk copy global -> shared with an L2 cache policy (createpolicy).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
 }
-// 16-byte async copy global -> shared; src_bytes = 0 fills zeros without reading.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-                 : "memory");
+// Streamed data (Phi, bit planes) is read once per step: evict it first.  The
+// expert directories are tiny and read by every CTA of every step: keep them.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-    return v;
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 // Shared load at a 32-bit shared address plus a constant byte offset.  Not
 // volatile, so the compiler may schedule it; its address always derives from a
-// descriptor loaded after the barrier that publishes the tables.
+// descriptor read after the barrier that publishes the tables.
 template <int OFF>
 __device__ __forceinline__ float lds_f32_imm(uint32_t addr) {
     float v;
     asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
     return v;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -141,241 +146,381 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
 __device__ __forceinline__ void red_add_release_u64(unsigned long long* p, unsigned long long v) {
     asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
+// Bounded spin until the grid-barrier counter reaches target; false on timeout.
+__device__ __forceinline__ bool grid_wait(const unsigned long long* ctr, unsigned long long target) {
+    if (ld_acquire_u64(ctr) >= target) return true;
+    const long long t0 = globaltimer();
+    while (ld_acquire_u64(ctr) < target)
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+    return true;
+}
 
 // ---------------------------------------------------------------------------
-// per-unit description (one routed (projection, slot) pair)
+// routed units and the column partition
 // ---------------------------------------------------------------------------
+// One routed (projection, slot) pair.
 struct UnitInfo {
-    int p, j, e;                 // projection, slot, expert (-1 when the id is out of range)
-    float g;                     // gate weight
-    int n16;                     // fp16 members
-    int pw;                      // plane words
-    int ntab;                    // nibble tables (8 per 32-member word)
-    uint32_t meta_off[kNumGroups];  // offsets of each group's metadata inside this unit's staging slot
-    uint32_t np[kNumGroups];     // padded members
-    uint32_t n[kNumGroups];      // members
-    uint32_t pw0[kNumGroups];    // first plane word of the group (bit-plane groups)
-    uint32_t tab0[kNumGroups];   // first table of the group
-    uint64_t planes_off[kNumGroups];  // byte offset of the group's planes in the blob
-    uint64_t w16_off;                 // byte offset of the fp16 rows in the blob
+    int p, j, e;  // projection, slot, expert (-1 when the id is out of range)
+    float g;      // gate weight
+    int pw;       // plane words
+    int n16;      // fp16 members
+    int items;    // plane words + octets of fp16 members
+    uint32_t np[kNumGroups], n[kNumGroups], pw0[kNumGroups];
+    uint64_t gbase[kNumGroups];  // byte offset of each group in the blob
 };
 
-__device__ inline void unit_info(const T1Params& P, int u, UnitInfo& U) {
+__device__ inline void unit_info(const T1Params& P, int u, int e, const uint8_t* s_dir, UnitInfo& U) {
     U.p = u / P.K;
     U.j = u % P.K;
-    int e = P.ids[U.j];
     U.e = (e >= 0 && e < P.E) ? e : -1;
     U.g = P.gw[U.j];
-    U.n16 = U.pw = U.ntab = 0;
-    uint32_t moff = 0, pw = 0, tab = 0;
-    if (U.e < 0) {
-        for (int g = 0; g < kNumGroups; g++) U.n[g] = U.np[g] = U.pw0[g] = U.tab0[g] = U.meta_off[g] = 0;
-        U.w16_off = 0;
-        return;
+    U.pw = U.n16 = U.items = 0;
+    for (int g = 0; g < kNumGroups; g++) {
+        U.np[g] = U.n[g] = U.pw0[g] = 0;
+        U.gbase[g] = 0;
     }
-    const uint8_t* blob = P.proj[U.p].blob;
-    const DirEntry d = read_dir(blob, U.e);
+    if (U.e < 0) return;
+    const DirEntry d = parse_dir(s_dir + ((size_t)U.p * P.E + U.e) * kDirEntryBytes);
+    uint32_t pw = 0;
     for (int g = 0; g < kNumGroups; g++) {
         const int b = group_width(g);
         U.n[g] = d.count[g];
         U.np[g] = (uint32_t)group_members_padded(b, d.count[g]);
-        U.meta_off[g] = moff;
         U.pw0[g] = pw;
-        U.tab0[g] = tab;
-        const uint64_t gbase = d.base + d.goff[g];
-        if (b == 16) {
-            moff += 6 * U.np[g];
-            U.w16_off = gbase + 6 * (uint64_t)U.np[g];
-            U.planes_off[g] = 0;
-        } else {
-            moff += 8 * U.np[g];
-            U.planes_off[g] = gbase + 8 * (uint64_t)U.np[g];
-            pw += (uint32_t)b * (U.np[g] / 32);
-            tab += U.np[g] / 4;
-        }
+        U.gbase[g] = d.base + d.goff[g];
+        if (b != 16) pw += (uint32_t)b * (U.np[g] / 32);
     }
-    U.n16 = (int)U.n[0];
     U.pw = (int)pw;
-    U.ntab = (int)tab;
+    U.n16 = (int)U.n[0];
+    U.items = U.pw + (U.n16 + kF16Item - 1) / kF16Item;
 }
 
-// Plane word q of a unit -> (group, bit plane, word).
+// Plane word q of a unit -> (group, bit plane, word).  Words are ordered by
+// group, then plane, then word.
 __device__ __forceinline__ void decode_pw(const UnitInfo& U, int q, int& g, int& jb, int& w) {
     g = 1;
 #pragma unroll
     for (int gg = 2; gg < kNumGroups; gg++)
-        if ((uint32_t)q >= U.pw0[gg]) g = gg;
+        if ((uint32_t)q >= U.pw0[gg] && U.np[gg] > 0) g = gg;
     const int W = (int)(U.np[g] / 32);
     const int rel = q - (int)U.pw0[g];
     jb = rel / W;
     w = rel - jb * W;
 }
 
-// Tasks [t0, t1) of a CTA.  With no more units than CTAs, every CTA works on
-// one unit only (units get floor or ceil of G/U CTAs, each a contiguous range
-// of the unit's row blocks), so each CTA builds one unit's tables; otherwise
-// the task list is cut into G contiguous pieces.
-__host__ __device__ inline void cta_tasks(const T1Params& P, int cta, int& t0, int& t1) {
-    const int U = 2 * P.K;
-    if (U <= P.G) {
-        const int u = (int)(((long long)cta * U) / P.G);
-        const int c0 = (int)(((long long)u * P.G + U - 1) / U), c1 = (int)(((long long)(u + 1) * P.G + U - 1) / U);
-        const int n = c1 - c0, i = cta - c0;
-        t0 = u * P.n_rb + (int)(((long long)i * P.n_rb) / n);
-        t1 = u * P.n_rb + (int)(((long long)(i + 1) * P.n_rb) / n);
-    } else {
-        t0 = (int)(((long long)cta * P.n_tasks) / P.G);
-        t1 = (int)(((long long)(cta + 1) * P.n_tasks) / P.G);
-    }
+// One work item of a CTA: a plane word (all rows of one bit plane of 32
+// members) or an octet of fp16 members (all rows).
+struct Item {
+    const uint8_t* ptr;  // plane word: its 32 words in tile 0; octet: member row 8f
+    uint32_t stride;     // plane word: bytes between the word's tiles
+    int16_t nf;          // octet: fp16 members in it (1..8); plane word: 0
+    int16_t slot;        // member-word slot (plane word) or octet slot
+    int16_t w;           // octet: f
+    int16_t u;           // unit
+};
+// A member word (32 members of a group) whose c values and tables this CTA builds.
+struct MemberWord {
+    const uint8_t* meta;  // the group's metadata: idx u16[np] | scale fp16[np] | amp f32[np]
+    uint32_t np;          // padded members of the group
+    int16_t p, g, w;
+    int16_t nvalid;  // real members in the word (0..32)
+    int16_t zp;      // 1 when this CTA evaluates the word's plane 0 and so owns its zero-point share
+    int16_t seg;
+};
+// Consecutive plane-word items of one group: contiguous in every 32-row tile,
+// so one bulk copy per tile stages all of them.
+struct Run {
+    const uint8_t* ptr;  // the first item's words in tile 0
+    uint32_t stride;     // bytes between tiles
+    int a, len;          // first item slot, items
+};
+// Items of one unit inside a CTA's share: plane words [i0, ip), fp16 octets [ip, i1).
+struct Seg {
+    int u, i0, ip, i1;
+};
+
+// Items [q0, q1) of CTA c out of Q: an equal contiguous share.  c * Q stays
+// below 2^32 for every shape the fused path takes (the host checks it).
+__host__ __device__ __forceinline__ int share_begin(int c, int Q, int G) {
+    return (int)(((uint32_t)c * (uint32_t)Q) / (uint32_t)G);
 }
 
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-// A run is a maximal set of consecutive tasks of this CTA that share a unit;
-// its staged plane words are laid out [plane word][rows of the run].
-struct RunInfo {
-    int ui;        // unit index inside the CTA
-    int t_first;   // first task
-    int nt;        // tasks in the run
-    int rows;      // staged rows (nt * kRB, clamped to d_pad)
-    uint32_t off;  // word offset of the run in the staging buffer
-};
-constexpr int kMaxRuns = kMaxUnitsPerCta;
-constexpr int kRunTasks = 4;  // tasks evaluated together (one accumulator each)
-
-__global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
+__global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t s_bar[kPhiBars + 1];  // Phi chunks, then planes + metadata
-    __shared__ UnitInfo s_unit[kMaxUnitsPerCta];
-    __shared__ RunInfo s_run[kMaxRuns];
-    __shared__ int s_abort, s_nruns;
+    __shared__ uint64_t s_bar[kPhiBars + 2];  // Phi chunks, the two expert directories, the staged planes
+    __shared__ Run s_run[kMaxItems];
+    __shared__ UnitInfo s_unit[kMaxUnits];
+    __shared__ Item s_item[kMaxItems];
+    __shared__ MemberWord s_mw[kMaxItems];
+    __shared__ Seg s_seg[kMaxItems];
+    __shared__ uint2 s_desc[kMaxItems];  // plane word: (tables' shared address, 2^j bits)
+    __shared__ float s_zpmw[kMaxItems];
+    __shared__ int s_ni, s_nmw, s_nseg, s_nrun, s_abort, s_bad;
+    __shared__ uint32_t s_stage_bytes;
     __shared__ unsigned long long s_bar_base;
-    __shared__ float s_zp;
-    __shared__ float s_zpw[kT1Warps];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nthreads = blockDim.x, nwarps = nthreads >> 5;
     const int cta = blockIdx.x;
-    int t0, t1;
-    cta_tasks(P, cta, t0, t1);
-    const int u_first = t0 / P.n_rb;
-    const int u_last = t1 > t0 ? (t1 - 1) / P.n_rb : u_first - 1;
-    const int nunits = u_last - u_first + 1;
-    const int rows_total = 2 * P.r;
-    const int row0 = (int)(((long long)cta * rows_total) / P.G);
-    const int row1 = (int)(((long long)(cta + 1) * rows_total) / P.G);
+    const int row0 = share_begin(cta, 2 * P.r, P.G), row1 = share_begin(cta + 1, 2 * P.r, P.G);
     const int nrows = row1 - row0;
     const uint32_t row_bytes = (uint32_t)P.d_in * 2;
 
     uint16_t* s_x = reinterpret_cast<uint16_t*>(smem + P.sm_x);
-    uint8_t* s_a = smem + P.sm_a;
-    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);
-    uint8_t* s_meta = smem + P.sm_meta;
+    uint8_t* s_dir = smem + P.sm_dir;  // [projection][expert] directory entries
+    uint8_t* s_phi = smem + P.sm_phi;
+    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);  // [tile][item slot][32]
+    uint8_t* s_mwd = smem + P.sm_mw;    // [member word]: idx u16[32] | scale u16[32] | amp f32[32]
+    uint8_t* s_f16d = smem + P.sm_f16;  // [octet]: idx u16[8] | amp f32[8]
+    float* s_c16 = reinterpret_cast<float*>(smem + P.sm_c16);  // [octet][8]
+    // tables start on a 512-byte shared-memory boundary: one member word's 8
+    // tables are 512 B, so the byte address of a word's tables has a zero low
+    // byte and a lookup can splice the entry offset into it with one byte permute
+    uint8_t* tab_raw = smem + P.sm_tab;
+    float* s_tab = reinterpret_cast<float*>(tab_raw + ((512u - (smem_u32(tab_raw) & 511u)) & 511u));
+    const uint32_t tab_sbase = smem_u32(s_tab);
 
-    // ---- phase 0: Phi rows and x first (they need nothing), by one thread ----
+    // ---- phase 0: the routed ids are loaded first; one thread initialises the
+    // mbarriers and then issues the Phi rows and x (they need nothing) ----
+    const int my_id = (warp == 1 && lane < P.U) ? P.ids[lane % P.K] : 0;
     if (tid == 0) {
-        for (int i = 0; i <= kPhiBars; i++) mbar_init(&s_bar[i], 1);
+        for (int i = 0; i < kPhiBars + 2; i++) mbar_init(&s_bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
         s_bar_base = ld_relaxed_u64(P.barrier);
+    }
+    __syncthreads();  // the mbarriers are initialised
+    if (tid == 0) {
+        // both expert directories first: the routed units need them before anything else
+        const uint32_t dir_bytes = (uint32_t)P.E * kDirEntryBytes;
+        const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+        mbar_expect_tx(&s_bar[kPhiBars], 2 * dir_bytes);
+        for (int p = 0; p < 2; p++)
+            bulk_g2s(s_dir + (size_t)p * dir_bytes, P.proj[p].blob + kHeaderBytes, dir_bytes, &s_bar[kPhiBars], keep);
         for (int bi = 0; bi < kPhiBars; bi++) {
             const int ra = row0 + (nrows * bi) / kPhiBars, rbnd = row0 + (nrows * (bi + 1)) / kPhiBars;
-            uint32_t bytes = (uint32_t)(rbnd - ra) * row_bytes + (bi == 0 ? row_bytes : 0);
+            const uint32_t bytes = (uint32_t)(rbnd - ra) * row_bytes + (bi == 0 ? row_bytes : 0);
             mbar_expect_tx(&s_bar[bi], bytes);
-            if (bi == 0) bulk_g2s(s_x, P.x, row_bytes, &s_bar[0]);
+            if (bi == 0) bulk_g2s(s_x, P.x, row_bytes, &s_bar[0], stream);
             for (int rr = ra; rr < rbnd;) {  // rows are contiguous inside a projection
                 const int p = rr / P.r, k = rr - p * P.r;
                 const int n = min(rbnd - rr, P.r - k);
-                bulk_g2s(s_a + (size_t)(rr - row0) * row_bytes, P.proj[p].phi_t + (size_t)k * P.d_in,
-                         (uint32_t)n * row_bytes, &s_bar[bi]);
+                bulk_g2s(s_phi + (size_t)(rr - row0) * row_bytes, P.proj[p].phi_t + (size_t)k * P.d_in,
+                         (uint32_t)n * row_bytes, &s_bar[bi], stream);
                 rr += n;
             }
         }
     }
-    // routed experts of this CTA's units (two dependent reads: ids, then the directory)
-    if (warp == 1 && lane < nunits) unit_info(P, u_first + lane, s_unit[lane]);
-    __syncthreads();  // s_unit ready
 
-    // runs of this CTA's tasks (one thread)
-    if (tid == 32) {
-        int nr = 0;
-        uint32_t off = 0;
-        for (int t = t0; t < t1;) {
-            const int ui = t / P.n_rb - u_first;
-            const int te = min(t1, (ui + u_first + 1) * P.n_rb);
-            while (t < te) {
-                const int nt = min(kRunTasks, te - t);
-                RunInfo R;
-                R.ui = ui;
-                R.t_first = t;
-                R.nt = nt;
-                R.rows = nt * kRB;
-                R.off = off;
-                const UnitInfo& U = s_unit[ui];
-                off += (uint32_t)(U.e >= 0 ? U.pw : 0) * (uint32_t)(nt * kRB);
-                s_run[nr++] = R;
-                t += nt;
+    // ---- routed units and this CTA's share (warp 1; one lane per unit, then per item).
+    // The other warps wait: this is short, and alone on the SM it is not slowed by them ----
+    if (warp == 1) {
+        const bool dir_ok = mbar_wait(&s_bar[kPhiBars], 0);
+        if (lane < P.U) unit_info(P, lane, dir_ok ? my_id : -1, s_dir, s_unit[lane]);
+        if (!dir_ok && lane == 0) s_abort = 1;
+        __syncwarp();
+        const bool is_unit = lane < P.U;
+        const int my_items = is_unit ? s_unit[lane].items : 0;
+        int incl = my_items;  // inclusive scan of items over units
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int excl = incl - my_items;
+        const int Q = __shfl_sync(0xffffffffu, incl, 31);
+        const int q0 = share_begin(cta, Q, P.G);
+        int ni = share_begin(cta + 1, Q, P.G) - q0;
+        if (ni > P.items_max || ni > kMaxItems) {  // the blob's counts disagree with the plan's
+            if (lane == 0 && P.status) atomicOr(P.status, BITSMOE_ST_PLANMISMATCH);
+            ni = 0;
+        }
+        const bool bad = __any_sync(0xffffffffu, is_unit && s_unit[lane].e < 0);
+        // unit of item `lane`: the number of units that end at or before it
+        int my_u = 0;
+#pragma unroll
+        for (int v = 0; v < 32; v++) my_u += (v < P.U && __shfl_sync(0xffffffffu, incl, v) <= q0 + lane) ? 1 : 0;
+        my_u = min(my_u, P.U - 1);
+        const int S_u = __shfl_sync(0xffffffffu, excl, my_u & 31);
+        const bool valid = lane < ni;
+        Item it{};
+        int key = -1 - lane, g = 0, jb = -1, w = 0;  // member-word key of a plane word; unique otherwise
+        if (valid) {
+            const UnitInfo& U = s_unit[my_u];
+            const int l = q0 + lane - S_u;
+            const uint8_t* blob = P.proj[U.p].blob;
+            it.u = (int16_t)my_u;
+            if (l < U.pw) {
+                decode_pw(U, l, g, jb, w);
+                const uint32_t b = (uint32_t)group_width(g), W = U.np[g] / 32;
+                it.ptr = blob + U.gbase[g] + 8ull * U.np[g] + 128ull * ((uint64_t)jb * W + (uint64_t)w);
+                it.stride = 128u * b * W;
+                it.nf = 0;
+                key = (my_u << 24) | (g << 16) | w;
+            } else {
+                const int f = l - U.pw;
+                it.ptr = blob + U.gbase[0] + 6ull * U.np[0] + 2ull * kF16Item * (uint64_t)f * (uint64_t)P.d_pad;
+                it.stride = 0;
+                it.nf = (int16_t)min(kF16Item, U.n16 - kF16Item * f);
+                it.w = (int16_t)f;
             }
         }
-        s_nruns = nr;
-        // bit planes (one copy per run, tile and group: the group's b x W x 32 words of a
-        // 32-row tile are contiguous) and per-component metadata (one copy per group)
-        uint32_t bytes = 0;
-        for (int ri = 0; ri < nr; ri++) {
-            const UnitInfo& U = s_unit[s_run[ri].ui];
-            if (U.e >= 0) bytes += 128u * (uint32_t)U.pw * (uint32_t)s_run[ri].nt;
-        }
-        for (int ui = 0; ui < nunits; ui++) {
-            const UnitInfo& U = s_unit[ui];
-            if (U.e < 0) continue;
-            for (int g = 0; g < kNumGroups; g++) bytes += (group_width(g) == 16 ? 6u : 8u) * U.np[g];
-        }
-        mbar_expect_tx(&s_bar[kPhiBars], bytes);
-        for (int ri = 0; ri < nr; ri++) {
-            const RunInfo& R = s_run[ri];
-            const UnitInfo& U = s_unit[R.ui];
-            if (U.e < 0) continue;
-            const uint8_t* blob = P.proj[U.p].blob;
-            const int tile0 = R.t_first % P.n_rb;
-            for (int k = 0; k < R.nt; k++)
-                for (int g = 1; g < kNumGroups; g++) {
-                    if (U.n[g] == 0) continue;
-                    const uint32_t gw = (uint32_t)group_width(g) * (U.np[g] / 32) * kRB;  // words per tile
-                    bulk_g2s(s_planes + R.off + (size_t)k * U.pw * kRB + (size_t)U.pw0[g] * kRB,
-                             blob + U.planes_off[g] + 4ull * gw * (uint64_t)(tile0 + k), 4u * gw, &s_bar[kPhiBars]);
-                }
-        }
-        for (int ui = 0; ui < nunits; ui++) {
-            const UnitInfo& U = s_unit[ui];
-            if (U.e < 0) continue;
-            const uint8_t* blob = P.proj[U.p].blob;
-            const DirEntry d = read_dir(blob, U.e);
-            for (int g = 0; g < kNumGroups; g++) {
-                if (U.n[g] == 0) continue;
-                bulk_g2s(s_meta + (size_t)ui * P.meta_max + U.meta_off[g], blob + d.base + d.goff[g],
-                         (group_width(g) == 16 ? 6u : 8u) * U.np[g], &s_bar[kPhiBars]);
+        const bool plane = valid && it.nf == 0, oct = valid && it.nf > 0;
+        // first item of the same member word, and whether any of them is plane 0
+        int ref = lane, zp = 0;
+        const int z0 = plane && jb == 0;
+#pragma unroll
+        for (int k = 0; k < 32; k++) {
+            const int kk = __shfl_sync(0xffffffffu, key, k), kz = __shfl_sync(0xffffffffu, z0, k);
+            if (k < ni && kk == key) {
+                if (k < ref) ref = k;
+                zp |= kz;
             }
+        }
+        const unsigned lt = (1u << lane) - 1u;
+        const bool newmw = plane && ref == lane;
+        const unsigned bm = __ballot_sync(0xffffffffu, newmw), bf = __ballot_sync(0xffffffffu, oct);
+        const int slot_new = __popc(bm & lt);
+        const int slot_ref = __shfl_sync(0xffffffffu, slot_new, ref);
+        const int slot = oct ? __popc(bf & lt) : slot_ref;
+        const int u_prev = __shfl_up_sync(0xffffffffu, my_u, 1);
+        const bool newseg = valid && (lane == 0 || u_prev != my_u);
+        const unsigned bs = __ballot_sync(0xffffffffu, newseg);
+        const int seg = __popc(bs & (lt | (1u << lane))) - 1;
+        if (valid) {
+            it.slot = (int16_t)slot;
+            s_item[lane] = it;
+            s_desc[lane] = plane ? make_uint2(tab_sbase + 512u * (uint32_t)slot, __float_as_uint((float)(1u << jb)))
+                                 : make_uint2(0u, 0u);
+        }
+        if (newmw) {
+            const UnitInfo& U = s_unit[my_u];
+            MemberWord M;
+            M.meta = P.proj[U.p].blob + U.gbase[g];
+            M.np = U.np[g];
+            M.p = (int16_t)U.p;
+            M.g = (int16_t)g;
+            M.w = (int16_t)w;
+            M.nvalid = (int16_t)max(0, min(32, (int)U.n[g] - 32 * w));
+            M.zp = (int16_t)zp;
+            M.seg = (int16_t)seg;
+            s_mw[slot_new] = M;
+        }
+        if (newseg) {
+            const unsigned above = bs & ~(lt | (1u << lane));
+            const int i1 = above ? __ffs(above) - 1 : ni;
+            const unsigned in_seg = (i1 >= 32 ? 0xffffffffu : ((1u << i1) - 1u)) & ~lt;
+            const unsigned octs = bf & in_seg;
+            Seg S;
+            S.u = my_u;
+            S.i0 = lane;
+            S.i1 = i1;
+            S.ip = octs ? __ffs(octs) - 1 : i1;
+            s_seg[seg] = S;
+        }
+        // runs of plane words: consecutive items whose words are contiguous in every tile
+        const uint64_t my_ptr = (uint64_t)it.ptr;
+        const uint64_t prev_ptr = __shfl_up_sync(0xffffffffu, my_ptr, 1);
+        const uint32_t prev_stride = __shfl_up_sync(0xffffffffu, it.stride, 1);
+        const int prev_plane = __shfl_up_sync(0xffffffffu, (int)plane, 1);
+        const bool cont = plane && lane > 0 && prev_plane && prev_stride == it.stride && my_ptr == prev_ptr + 128u;
+        const unsigned bcont = __ballot_sync(0xffffffffu, cont), bplane = __ballot_sync(0xffffffffu, plane);
+        const unsigned brun = bplane & ~bcont;
+        if ((brun >> lane) & 1u) {
+            const unsigned stop = ~bcont & (lane == 31 ? 0u : ~((2u << lane) - 1u));  // first later item not continuing
+            Run R;
+            R.ptr = it.ptr;
+            R.stride = it.stride;
+            R.a = lane;
+            R.len = (stop ? __ffs(stop) - 1 : 32) - lane;
+            s_run[__popc(brun & lt)] = R;
+        }
+        if (lane == 0) {
+            s_ni = ni;
+            s_nmw = __popc(bm);
+            s_nseg = __popc(bs);
+            s_nrun = __popc(brun);
+            s_stage_bytes = 128u * (uint32_t)__popc(bplane) * (uint32_t)P.n_rb + 256u * __popc(bm) + 48u * __popc(bf);
+            s_bad = bad;
+        }
+    }
+    __syncthreads();
+    const int ni = s_ni, nmw = s_nmw, nseg = s_nseg;
+    // The last kStageWarps warps issue the staging copies; their issue can stall
+    // behind the Phi traffic, so the z rows are left to the other warps.
+    const int nrw = nwarps - kStageWarps;  // row warps
+    const bool row_warp = warp < nrw;
+
+    // ---- the outputs are sums of red.add contributions: each CTA zeroes a slice first ----
+    {
+        const int nys = 2 * P.d_out;
+        const int nye0 = P.proj[0].Ye ? P.K * P.d_out : 0, nye1 = P.proj[1].Ye ? P.K * P.d_out : 0;
+        const int tot = nys + nye0 + nye1;
+        const int a = share_begin(cta, tot, P.G), b = share_begin(cta + 1, tot, P.G);
+        for (int i = a + tid; row_warp && i < b; i += nrw * 32) {
+            float* dst;
+            if (i < P.d_out)
+                dst = P.proj[0].Ysum + i;
+            else if (i < nys)
+                dst = P.proj[1].Ysum + (i - P.d_out);
+            else if (i < nys + nye0)
+                dst = P.proj[0].Ye + (i - nys);
+            else
+                dst = P.proj[1].Ye + (i - nys - nye0);
+            *dst = 0.0f;
         }
     }
 
-    // ---- phase 1: z rows of this CTA on every warp but warp 1 (which issues the plane copies) ----
-    // The grid barrier is split: thread 0 arrives as soon as the row warps are
-    // done (named barrier 1), and waits only after that.  The counter is a
-    // multiple of G whenever no launch is in flight (it starts at zero and every
-    // launch adds exactly G), so the value read at start rounded down to a
-    // multiple of G is this launch's base.
-    if (warp != 1) {
-        const int wv = warp == 0 ? kT1Warps - 2 : warp - 2;  // 0 .. kT1Warps-2
-        constexpr int kRowWarps = kT1Warps - 1;
+    // ---- staging by the staging warp (bulk copies on one mbarrier): plane-word runs
+    // into [tile][item slot], one copy per run and tile; then each member word's idx,
+    // scale and amp, and each octet's idx and amp ----
+    if (!row_warp) {
+        const int st = threadIdx.x - nrw * 32, nst = kStageWarps * 32;
+        const uint64_t stream = policy_evict_first();
+        uint64_t* bar = &s_bar[kPhiBars + 1];
+        if (st == 0) mbar_expect_tx(bar, s_stage_bytes);
+        __syncwarp();
+        const uint32_t tstride = 128u * (uint32_t)P.items_max;  // bytes between tiles in s_planes
+        const int nr = s_nrun;
+        for (int pr = st; pr < nr * P.n_rb; pr += nst) {
+            const int r = pr / P.n_rb, t = pr - r * P.n_rb;
+            const Run R = s_run[r];
+            bulk_g2s(reinterpret_cast<uint8_t*>(s_planes) + (size_t)t * tstride + 128u * R.a,
+                     R.ptr + (uint64_t)t * R.stride, 128u * (uint32_t)R.len, bar, stream);
+        }
+        for (int m = st; m < nmw; m += nst) {
+            const MemberWord& M = s_mw[m];
+            uint8_t* dst = s_mwd + 256 * m;
+            bulk_g2s(dst, M.meta + 64ull * M.w, 64u, bar, stream);                              // idx
+            bulk_g2s(dst + 64, M.meta + 2ull * M.np + 64ull * M.w, 64u, bar, stream);            // scale
+            bulk_g2s(dst + 128, M.meta + 4ull * M.np + 128ull * M.w, 128u, bar, stream);         // amp
+        }
+        for (int i = st; i < ni; i += nst) {
+            const Item& it = s_item[i];
+            if (!it.nf) continue;
+            const UnitInfo& U = s_unit[it.u];
+            const uint8_t* gb = P.proj[U.p].blob + U.gbase[0];
+            uint8_t* dst = s_f16d + 48 * it.slot;
+            bulk_g2s(dst, gb + 16ull * it.w, 16u, bar, stream);
+            bulk_g2s(dst + 16, gb + 2ull * U.np[0] + 32ull * it.w, 32u, bar, stream);
+        }
+    }
+
+    // ---- phase 1: z rows of this CTA (row warps), then the arrival at the grid barrier ----
+    const unsigned long long G = (unsigned long long)P.G;
+    if (row_warp) {
         bool ok = nrows == 0 || mbar_wait(&s_bar[0], 0);  // barrier 0 carries x
-        for (int rl = wv; ok && rl < nrows; rl += kRowWarps) {
+        for (int rl = warp; ok && rl < nrows; rl += nrw) {
             int bi = 0;
             while (bi + 1 < kPhiBars && rl >= (nrows * (bi + 1)) / kPhiBars) bi++;
             if (!mbar_wait(&s_bar[bi], 0)) {
                 ok = false;
                 break;
             }
-            const uint4* rowv = reinterpret_cast<const uint4*>(s_a + (size_t)rl * row_bytes);
+            const uint4* rowv = reinterpret_cast<const uint4*>(s_phi + (size_t)rl * row_bytes);
             const uint4* xv = reinterpret_cast<const uint4*>(s_x);
             float acc = 0.0f;
             for (int i8 = lane; i8 < P.d_in / 8; i8 += 32) {
@@ -397,219 +542,117 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
             }
         }
         if (!ok) s_abort = 1;
-        asm volatile("bar.sync 1, %0;" ::"n"(kRowWarps * 32) : "memory");
+        // The row warps' z rows and zeroed outputs are ordered before the arrival by
+        // this CTA barrier and the cumulative release of the arrival itself.
+        asm volatile("bar.sync 1, %0;" ::"r"(nrw * 32) : "memory");
         if (tid == 0) {
-            // every bulk copy of Phi into this CTA's shared memory has landed (bounded)
-            for (int bi = 0; bi < kPhiBars; bi++)
+            for (int bi = 0; bi < kPhiBars; bi++)  // every bulk copy into this CTA's shared memory has landed
                 if (!mbar_wait(&s_bar[bi], 0)) s_abort = 1;
+            __threadfence();
             red_add_release_u64(P.barrier, 1ull);  // arrive
         }
     }
-    __syncthreads();  // warp 1 has issued its copies; s_run is visible
+    __syncthreads();
 
-    // ---- grid barrier wait (bounded), then the planes ----
+    // ---- grid barrier wait (bounded) ----
+    // The counter is a multiple of G whenever no launch is in flight (it starts
+    // at zero and every launch adds exactly G), so the value read at start
+    // rounded down to a multiple of G is this launch's base.
+    const unsigned long long base = (s_bar_base / G) * G;
     if (tid == 0) {
-        const unsigned long long G = (unsigned long long)P.G;
-        const unsigned long long target = (s_bar_base / G + 1) * G;
-        if (ld_acquire_u64(P.barrier) < target) {
-            const long long tw = globaltimer();
-            while (ld_acquire_u64(P.barrier) < target) {
-                if (globaltimer() - tw > kWaitLimitNs) {
-                    s_abort = 1;
-                    break;
-                }
-            }
-        }
-        if (!mbar_wait(&s_bar[kPhiBars], 0)) s_abort = 1;  // planes and metadata
-        if (s_abort && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
+        if (!grid_wait(P.barrier, base + G)) s_abort = 1;
+        if (!mbar_wait(&s_bar[kPhiBars + 1], 0)) s_abort = 1;  // the staged planes and metadata
+        if (s_bad && cta == 0 && P.status) atomicOr(P.status, BITSMOE_ST_BADEXPERT);
     }
     __syncthreads();
-    if (s_abort) return;
+    if (s_abort) {
+        if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
+        return;
+    }
 
-    // ---- phase 2: z of the needed projections, then the runs ----
-    float* s_z = reinterpret_cast<float*>(s_a + P.a_z);
-    // tables start on a 512-byte shared-memory boundary: one word's 8 tables are 512 B, so the
-    // byte address of a word's tables has a zero low byte and a lookup can splice the entry
-    // offset into it with one byte permute
-    float* s_tab = reinterpret_cast<float*>(s_a + P.a_tab + ((512u - (smem_u32(s_a + P.a_tab) & 511u)) & 511u));
-    float* s_part = reinterpret_cast<float*>(s_a + P.a_part);
-    float* s_c16 = reinterpret_cast<float*>(s_a + P.a_c16);
-    uint2* s_desc = reinterpret_cast<uint2*>(s_a + P.a_desc);
-    float* s_cm = reinterpret_cast<float*>(s_a + P.a_cm);
-    const uint32_t tab_sbase = smem_u32(s_tab);
-    {
-        bool need[2] = {false, false};
-        for (int ui = 0; ui < nunits; ui++) need[s_unit[ui].p] = true;
-        for (int p = 0; p < 2; p++)
-            if (need[p])
-                for (int i = tid; i < P.r; i += kT1Threads) s_z[p * P.r + i] = __ldcg(P.zbuf + p * P.r + i);
+    // ---- c_k = a_k s_k z_k, the tables and the zero-point share: a warp per member word ----
+    for (int m = warp; m < nmw; m += nwarps) {
+        const MemberWord M = s_mw[m];
+        const uint8_t* md = s_mwd + 256 * m;
+        const int k = reinterpret_cast<const uint16_t*>(md)[lane];
+        float c = 0.0f;
+        if (lane < M.nvalid && k < P.r)
+            c = reinterpret_cast<const float*>(md + 128)[lane] *
+                __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(md + 64)[lane])) *
+                __ldcg(P.zbuf + M.p * P.r + k);
+        // entry e of table tb = the sum of c over the set bits of e (members 4 tb .. 4 tb + 3)
+        const int e = lane & 15;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const int tb = (lane >> 4) + 2 * q;
+            const float c0 = __shfl_sync(0xffffffffu, c, 4 * tb), c1 = __shfl_sync(0xffffffffu, c, 4 * tb + 1);
+            const float c2 = __shfl_sync(0xffffffffu, c, 4 * tb + 2), c3 = __shfl_sync(0xffffffffu, c, 4 * tb + 3);
+            s_tab[128 * m + 16 * tb + e] =
+                ((e & 1 ? c0 : 0.0f) + (e & 2 ? c1 : 0.0f)) + ((e & 4 ? c2 : 0.0f) + (e & 8 ? c3 : 0.0f));
+        }
+        float h = M.zp ? 0.5f * (float)((1 << group_width(M.g)) - 1) * c : 0.0f;
+        h = warp_sum(h);
+        if (lane == 0) s_zpmw[m] = h;
+    }
+    for (int ch = tid; ch < ni * kF16Item; ch += nthreads) {
+        const int i = ch / kF16Item, m = ch - i * kF16Item;
+        const Item& it = s_item[i];
+        if (!it.nf) continue;
+        const uint8_t* fd = s_f16d + 48 * it.slot;
+        const int k = reinterpret_cast<const uint16_t*>(fd)[m];
+        float c = 0.0f;
+        if (m < it.nf && k < P.r)
+            c = reinterpret_cast<const float*>(fd + 16)[m] * __ldcg(P.zbuf + s_unit[it.u].p * P.r + k);
+        s_c16[kF16Item * it.slot + m] = c;
     }
     __syncthreads();
-    int cur_unit = -1;
-    const int nruns = s_nruns;
-    for (int ri = 0; ri < nruns; ri++) {
-        const RunInfo R = s_run[ri];
-        const UnitInfo& U = s_unit[R.ui];
-        if (R.ui != cur_unit && U.e >= 0) {
-            __syncthreads();  // the previous unit's tables and descriptors are no longer read
-            const uint8_t* meta = s_meta + (size_t)R.ui * P.meta_max;
-            const float* z = s_z + U.p * P.r;
-            float zp = 0.0f;
-            // pass 1: c_k = a_k s_k z_k of every member (bit-plane groups, concatenated in
-            // group order and padded: member m of table tb is 4 tb + (m % 4)), and the
-            // zero-point partial sums.  Group fields are copied to registers first: the
-            // stores below go to shared memory, where UnitInfo also lives.
-            for (int g = 1; g < kNumGroups; g++) {
-                const uint32_t np = U.np[g], n = U.n[g], m0 = 4 * U.tab0[g];
-                if (np == 0) continue;
-                const uint8_t* gm = meta + U.meta_off[g];
-                const float* __restrict__ amp = reinterpret_cast<const float*>(gm + 4 * np);
-                const uint16_t* __restrict__ scl = reinterpret_cast<const uint16_t*>(gm + 2 * np);
-                const uint16_t* __restrict__ idx = reinterpret_cast<const uint16_t*>(gm);
-                const float hr = 0.5f * (float)((1 << group_width(g)) - 1);
-                for (uint32_t ml = tid; ml < np; ml += kT1Threads) {
-                    float c = 0.0f;
-                    if (ml < n) c = amp[ml] * __half2float(__ushort_as_half(scl[ml])) * z[idx[ml]];
-                    s_cm[m0 + ml] = c;
-                    zp += hr * c;
-                }
+
+    // ---- lookups: warps own 32-row tiles; a segment's rows go to Y_e and, times g, to Y_sum ----
+    for (int s = 0; s < nseg; s++) {
+        const Seg S = s_seg[s];
+        const UnitInfo& U = s_unit[S.u];
+        const int p = U.p;
+        float* ye = P.proj[p].Ye ? P.proj[p].Ye + (size_t)U.j * P.d_out : nullptr;
+        float* ys = P.proj[p].Ysum;
+        const float gj = U.g;
+        // this CTA's zero-point share of the unit (member words in slot order)
+        const float zps = warp_sum(lane < nmw && s_mw[lane].seg == s ? s_zpmw[lane] : 0.0f);
+        for (int t = warp; t < P.n_rb; t += nwarps) {
+            const uint32_t* pl = s_planes + (size_t)t * P.items_max * kRB + lane;  // [tile][item slot][32]
+            float acc = 0.0f;
+#pragma unroll 2
+            for (int i = S.i0; i < S.ip; i++) {
+                const uint2 d = s_desc[i];
+                const uint32_t word = pl[i * kRB];
+                // entry offsets (nibble x 4 bytes): even nibbles in the bytes of lo, odd in hi;
+                // table n of this word is at d.x + 64 n, entry e at + 4 e
+                const uint32_t lo = (word << 2) & 0x3C3C3C3Cu, hi = (word >> 2) & 0x3C3C3C3Cu;
+                float l[8];
+                l[0] = lds_f32_imm<0>(__byte_perm(lo, d.x, 0x7650u));
+                l[1] = lds_f32_imm<64>(__byte_perm(hi, d.x, 0x7650u));
+                l[2] = lds_f32_imm<128>(__byte_perm(lo, d.x, 0x7651u));
+                l[3] = lds_f32_imm<192>(__byte_perm(hi, d.x, 0x7651u));
+                l[4] = lds_f32_imm<256>(__byte_perm(lo, d.x, 0x7652u));
+                l[5] = lds_f32_imm<320>(__byte_perm(hi, d.x, 0x7652u));
+                l[6] = lds_f32_imm<384>(__byte_perm(lo, d.x, 0x7653u));
+                l[7] = lds_f32_imm<448>(__byte_perm(hi, d.x, 0x7653u));
+                const float sum = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
+                acc = fmaf(sum, __uint_as_float(d.y), acc);
             }
-            __syncthreads();
-            // pass 2: entry n of table tb = sum of c over the set bits of n (one entry per
-            // thread and step; four steps' loads are issued before their stores)
-            {
-                const int nent = 16 * U.ntab;
-                const float4* __restrict__ cm4 = reinterpret_cast<const float4*>(s_cm);
-                float* __restrict__ tab = s_tab;
-                const int n = tid & 15;  // kT1Threads is a multiple of 16: n is fixed per thread
-                for (int en0 = tid; en0 < nent; en0 += 4 * kT1Threads) {
-                    float4 c4[4];
-#pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const int en = en0 + u * kT1Threads;
-                        c4[u] = en < nent ? cm4[en >> 4] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const int en = en0 + u * kT1Threads;
-                        if (en < nent)
-                            tab[en] = ((n & 1 ? c4[u].x : 0.0f) + (n & 2 ? c4[u].y : 0.0f)) +
-                                      ((n & 4 ? c4[u].z : 0.0f) + (n & 8 ? c4[u].w : 0.0f));
-                    }
-                }
-            }
-            // plane-word descriptors: shared-memory byte offset of the word's 8 tables, weight 2^j
-            for (int q = tid; q < U.pw; q += kT1Threads) {
-                int g, jb, w;
-                decode_pw(U, q, g, jb, w);
-                s_desc[q] = make_uint2(tab_sbase + 64u * (U.tab0[g] + 8u * (uint32_t)w), __float_as_uint((float)(1u << jb)));
-            }
-            if (U.n16 > 0) {
-                const uint8_t* gm = meta + U.meta_off[0];
-                const uint16_t* idx = reinterpret_cast<const uint16_t*>(gm);
-                const float* amp = reinterpret_cast<const float*>(gm + 2 * U.np[0]);
-                for (int m = tid; m < U.n16; m += kT1Threads) s_c16[m] = amp[m] * z[idx[m]];
-            }
-            zp = warp_sum(zp);
-            if (lane == 0) s_zpw[warp] = zp;
-            __syncthreads();
-            if (warp == 0) {
-                float v = lane < kT1Warps ? s_zpw[lane] : 0.0f;
-                v = warp_sum(v);
-                if (lane == 0) s_zp = v;
-            }
-            __syncthreads();
-            cur_unit = R.ui;
-        }
-        // every warp takes a share of the unit's plane words for all tasks of the run
-        float acc[kRunTasks];
-#pragma unroll
-        for (int k = 0; k < kRunTasks; k++) acc[k] = 0.0f;
-        if (U.e >= 0) {
-            const int stride = U.pw * kRB;  // words between consecutive tasks (tiles) of the run
-            const uint32_t* pl = s_planes + R.off + lane;
-            for (int q = warp; q < U.pw; q += kT1Warps) {
-                const uint2 d = s_desc[q];
-                const float wt = __uint_as_float(d.y);
-#pragma unroll
-                for (int k = 0; k < kRunTasks; k++) {
-                    if (k < R.nt) {
-                        const uint32_t word = pl[k * stride + q * kRB];
-                        // entry offsets (nibble x 4 bytes): even nibbles in the bytes of lo, odd in hi;
-                        // table n of this word is at d.x + 64 n, entry e at + 4 e
-                        const uint32_t lo = (word << 2) & 0x3C3C3C3Cu, hi = (word >> 2) & 0x3C3C3C3Cu;
-                        float l[8];
-                        l[0] = lds_f32_imm<0>(__byte_perm(lo, d.x, 0x7650u));
-                        l[1] = lds_f32_imm<64>(__byte_perm(hi, d.x, 0x7650u));
-                        l[2] = lds_f32_imm<128>(__byte_perm(lo, d.x, 0x7651u));
-                        l[3] = lds_f32_imm<192>(__byte_perm(hi, d.x, 0x7651u));
-                        l[4] = lds_f32_imm<256>(__byte_perm(lo, d.x, 0x7652u));
-                        l[5] = lds_f32_imm<320>(__byte_perm(hi, d.x, 0x7652u));
-                        l[6] = lds_f32_imm<384>(__byte_perm(lo, d.x, 0x7653u));
-                        l[7] = lds_f32_imm<448>(__byte_perm(hi, d.x, 0x7653u));
-                        const float sum = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
-                        acc[k] = fmaf(sum, wt, acc[k]);
-                    }
-                }
-            }
-            if (U.n16 > 0) {
-                const uint16_t* w16 = reinterpret_cast<const uint16_t*>(P.proj[U.p].blob + U.w16_off);
-#pragma unroll
-                for (int k = 0; k < kRunTasks; k++) {
-                    const int row = ((R.t_first + k) % P.n_rb) * kRB + lane;
-                    if (k < R.nt && row < P.d_out)
-                        for (int m = warp; m < U.n16; m += kT1Warps)
-                            acc[k] = fmaf(s_c16[m], __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row])),
-                                          acc[k]);
-                }
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < kRunTasks; k++) s_part[(k * kT1Warps + warp) * kRB + lane] = acc[k];
-        __syncthreads();
-        if (warp < R.nt) {  // warp k reduces task k of the run
-            const int k = warp, t = R.t_first + k, rb = t % P.n_rb, row = rb * kRB + lane;
-            float y = 0.0f;
-            if (U.e >= 0) {
-#pragma unroll
-                for (int w = 0; w < kT1Warps; w++) y += s_part[(k * kT1Warps + w) * kRB + lane];
-                y -= s_zp;
+            const int row = t * kRB + lane;
+            for (int i = S.ip; i < S.i1; i++) {  // fp16 octets, rows read in place
+                const Item& it = s_item[i];
+                const uint16_t* w16 = reinterpret_cast<const uint16_t*>(it.ptr);
+                for (int m = 0; m < it.nf; m++)
+                    acc = fmaf(s_c16[kF16Item * it.slot + m],
+                               __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row])), acc);
             }
             if (row < P.d_out) {
-                if (P.proj[U.p].Ye) P.proj[U.p].Ye[(size_t)U.j * P.d_out + row] = y;
-                P.scratch[((size_t)U.p * P.K + U.j) * P.d_pad + row] = U.e >= 0 ? U.g * y : 0.0f;
+                const float y = acc - zps;
+                if (ye) red_add_f32(ye + row, y);
+                red_add_f32(ys + row, gj * y);
             }
         }
-        __syncthreads();
-    }
-    // ordered routed sum: every task of this CTA is published with one fence, its
-    // row-block counters bumped together, and the last slot of a row block sums
-    // the K weighted rows in slot order.
-    __threadfence();
-    __syncthreads();
-    __shared__ uint32_t s_last[64];
-    const int ntask = t1 - t0;
-    for (int i = tid; i < ntask; i += kT1Threads) {
-        const int t = t0 + i, p = (t / P.n_rb) / P.K, rb = t % P.n_rb;
-        const uint32_t old = atomicAdd(&P.rb_count[p * P.n_rb + rb], 1u);
-        s_last[i] = old == (uint32_t)(P.K - 1);
-    }
-    __syncthreads();
-    __threadfence();
-    for (int i = warp; i < ntask; i += kT1Warps) {
-        if (!s_last[i]) continue;
-        const int t = t0 + i, p = (t / P.n_rb) / P.K, rb = t % P.n_rb;
-        const int row = rb * kRB + lane;
-        if (row < P.d_out) {
-            float s = 0.0f;
-            for (int j = 0; j < P.K; j++) s += __ldcg(P.scratch + ((size_t)p * P.K + j) * P.d_pad + row);
-            P.proj[p].Ysum[row] = s;
-        }
-        if (lane == 0) P.rb_count[p * P.n_rb + rb] = 0u;
-    }
-    if (tid == 0 && P.status) {
-        for (int ui = 0; ui < nunits; ui++)
-            if (s_unit[ui].e < 0) atomicOr(P.status, BITSMOE_ST_BADEXPERT);
     }
 }
 
@@ -619,43 +662,57 @@ __global__ void __launch_bounds__(kT1Threads, 1) k_layer_t1(const T1Params P) {
 struct T1Layout {
     bool ok;
     T1Params P;
-    uint64_t ws_reserved;  // persistent counters at the start of the workspace
+    uint64_t ws_reserved;  // persistent counter at the start of the workspace
     uint64_t ws_bytes;
     size_t smem;
+    int threads;
 };
 
 static int g_num_sms = 0;
 static int g_max_smem = 0;
+static int g_static_smem = -1;
 
 static bool device_info() {
-    if (g_num_sms > 0) return true;
+    if (g_num_sms > 0 && g_static_smem >= 0) return true;
     int dev;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     if (cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
     if (cudaDeviceGetAttribute(&g_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k_layer_t1) != cudaSuccess) return false;
+    g_static_smem = (int)fa.sharedSizeBytes;
     return true;
 }
 
-static void unit_bounds(const bitsmoe_plan* p, int& pw, int& members, int& meta, int& n16) {
+// Work items (plane words + fp16 octets) of the largest expert of a plan.
+static int expert_items_max(const bitsmoe_plan* p) {
+    int best = 0;
     for (int e = 0; e < p->dims.n_experts; e++) {
         const uint32_t* c = p->counts + 8 * (size_t)e;
-        int w = 0, m = 0, mb = 0;
+        int pw = 0;
         for (int g = 0; g < kNumGroups; g++) {
             const int b = group_width(g);
-            const int np = (int)group_members_padded(b, c[g]);
-            if (b == 16) {
-                mb += 6 * np;
-            } else {
-                mb += 8 * np;
-                m += np;
-                w += b * (np / 32);
-            }
+            if (b != 16) pw += b * (int)(group_members_padded(b, c[g]) / 32);
         }
-        pw = std::max(pw, w);
-        members = std::max(members, m);
-        meta = std::max(meta, mb);
-        n16 = std::max(n16, (int)c[0]);
+        best = std::max(best, pw + (int)((c[0] + kF16Item - 1) / kF16Item));
     }
+    return best;
+}
+
+// Warps per CTA: every warp owns whole 32-row tiles, so take the count (8..24)
+// that leaves the fewest idle warp-tiles, the larger on a tie.
+static int choose_warps(int n_rb) {
+    int best = 8;
+    double best_eff = 0.0;
+    for (int nw = 8; nw <= kT1MaxWarps; nw++) {
+        const int per = (n_rb + nw - 1) / nw;
+        const double eff = (double)n_rb / (double)(per * nw);
+        if (eff >= best_eff) {
+            best_eff = eff;
+            best = nw;
+        }
+    }
+    return best;
 }
 
 static uint32_t align_up(uint64_t v, uint64_t a) { return (uint32_t)roundup(v, a); }
@@ -672,51 +729,34 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     P.r = g->dims.rank;
     P.K = g->dims.top_k;
     P.E = g->dims.n_experts;
-    if (u->dims.d_out != P.d_out || u->dims.rank != P.r) return L;
+    P.U = 2 * P.K;
+    if (u->dims.d_out != P.d_out || u->dims.rank != P.r || u->dims.d_in != P.d_in) return L;
+    if (P.U > kMaxUnits || P.d_in % 8 || P.d_in > 8192 || P.d_pad % kRB) return L;
     P.G = g_num_sms;
-    P.n_rb = (P.d_out + kRB - 1) / kRB;
-    P.n_tasks = 2 * P.K * P.n_rb;
-    P.phi_rows = (2 * P.r + P.G - 1) / P.G;
-    P.tasks_max = 0;
-    int units_max = 0;
-    for (int c = 0; c < P.G; c++) {  // exact bounds of the partition the kernel uses
-        int a, b;
-        cta_tasks(P, c, a, b);
-        P.tasks_max = std::max(P.tasks_max, b - a);
-        if (b > a) units_max = std::max(units_max, (b - 1) / P.n_rb - a / P.n_rb + 1);
-    }
-    int pw = 0, members = 0, meta = 0, n16 = 0;
-    unit_bounds(g, pw, members, meta, n16);
-    unit_bounds(u, pw, members, meta, n16);
-    P.pw_max = pw;
-    P.members_max = members;
-    P.meta_max = align_up(meta, 16);
-    P.n16_max = n16;
-
-    if (units_max > kMaxUnitsPerCta || P.tasks_max > 64 || P.d_in % 8 || P.d_in > 8192) return L;
-    if (units_max + (P.tasks_max + kRunTasks - 1) / kRunTasks > kMaxRuns) return L;
-    // shared memory
-    const uint64_t phi_bytes = (uint64_t)P.phi_rows * P.d_in * 2;
-    P.a_z = 0;
-    P.a_tab = align_up(P.a_z + 8ull * P.r, 128);
-    P.a_part = align_up(P.a_tab + 512 + 16ull * 4 * (members / 4), 16);  // + 512: tables realigned in the kernel
-    P.a_c16 = align_up(P.a_part + 4ull * kRunTasks * kT1Warps * kRB, 16);
-    P.a_desc = align_up(P.a_c16 + 4ull * n16, 16);
-    P.a_cm = align_up(P.a_desc + 8ull * P.pw_max, 16);
-    const uint64_t a_bytes = std::max<uint64_t>(phi_bytes, P.a_cm + 4ull * members);
+    P.n_rb = P.d_pad / kRB;
+    const long long q_max = (long long)P.K * (expert_items_max(g) + expert_items_max(u));
+    P.items_max = (int)((q_max + P.G - 1) / P.G);
+    if (P.items_max > kMaxItems) return L;
+    if ((uint64_t)P.G * (uint64_t)std::max<long long>(q_max, 2ll * std::max(P.r, P.d_out) * (P.K + 1)) >= (1ull << 32))
+        return L;  // the 32-bit share arithmetic
+    if (2ull * kDirEntryBytes * P.E >= (1u << 20)) return L;  // one mbarrier transaction count
+    const int im = std::max(1, P.items_max);
+    const int phi_rows = (2 * P.r + P.G - 1) / P.G;
     P.sm_x = 0;
-    P.sm_a = align_up(P.sm_x + 2ull * P.d_in, 128);
-    P.sm_planes = align_up(P.sm_a + a_bytes, 128);
-    P.sm_meta = align_up(P.sm_planes + 4ull * kRB * P.pw_max * P.tasks_max, 128);
-    P.sm_end = align_up(P.sm_meta + (uint64_t)P.meta_max * units_max, 128);
+    P.sm_dir = align_up(2ull * P.d_in, 128);
+    P.sm_phi = align_up(P.sm_dir + 2ull * kDirEntryBytes * P.E, 128);
+    P.sm_planes = align_up(P.sm_phi + (uint64_t)phi_rows * P.d_in * 2, 128);
+    P.sm_mw = align_up(P.sm_planes + 128ull * P.n_rb * im, 128);
+    P.sm_f16 = align_up(P.sm_mw + 256ull * im, 16);
+    P.sm_c16 = align_up(P.sm_f16 + 48ull * im, 16);
+    P.sm_tab = align_up(P.sm_c16 + 32ull * im, 16);
+    P.sm_end = align_up(P.sm_tab + 512ull + 512ull * im, 16);  // + 512: tables realigned in the kernel
     L.smem = P.sm_end;
-    const size_t static_smem = sizeof(uint64_t) * kPhiBars + sizeof(UnitInfo) * kMaxUnitsPerCta + 256;
-    if (L.smem + static_smem > (size_t)g_max_smem) return L;
-    // workspace: [barrier | rb_count] persistent at the head, then zbuf and scratch
-    L.ws_reserved = roundup(256 + 4ull * 2 * P.n_rb, 256);
-    uint64_t off = roundup(4ull * 2 * P.r, 256);
-    off = roundup(off + 4ull * 2 * P.K * P.d_pad, 256);
-    L.ws_bytes = off;  // bytes after the reserved head
+    if (L.smem + (size_t)g_static_smem > (size_t)g_max_smem) return L;
+    L.threads = 32 * choose_warps(P.n_rb);
+    // workspace: [barrier counter] persistent at the head, then z
+    L.ws_reserved = 256;
+    L.ws_bytes = roundup(4ull * 2 * P.r, 256);  // bytes after the reserved head
     L.ok = true;
     return L;
 }
@@ -728,7 +768,7 @@ uint64_t layer_fused_t1_workspace(const bitsmoe_plan* g, const bitsmoe_plan* u) 
 }
 
 // Bytes at the head of a layer workspace that hold the fused path's
-// persistent counters (0 when it does not apply).
+// persistent counter (0 when it does not apply).
 uint64_t layer_fused_t1_reserved(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     T1Layout L = t1_layout(g, u);
     return L.ok ? L.ws_reserved : 0;
@@ -753,17 +793,13 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
     P.status = status;
     uint8_t* ws = (uint8_t*)workspace;
     P.barrier = (unsigned long long*)ws;
-    P.rb_count = (uint32_t*)(ws + 256);
-    uint64_t off = L.ws_reserved;
-    P.zbuf = (float*)(ws + off);
-    off = roundup(off + 4ull * 2 * P.r, 256);
-    P.scratch = (float*)(ws + off);
+    P.zbuf = (float*)(ws + L.ws_reserved);
 
     cudaError_t e = cudaFuncSetAttribute(k_layer_t1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
     if (e != cudaSuccess) return set_cuda_error(e);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)P.G);
-    cfg.blockDim = dim3(kT1Threads);
+    cfg.blockDim = dim3((unsigned)L.threads);
     cfg.dynamicSmemBytes = L.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -782,8 +818,8 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
 // ---------------------------------------------------------------------------
 // Single-token layer forward with library-owned scratch, for callers that
 // cannot allocate device memory.  The scratch (the fused kernel's grid-barrier
-// counter, row-block counters, z of both projections and the weighted rows of
-// the routed sum) lives in one fixed static device array instead of a
+// counter, z of both projections and the partial rows of the routed sum)
+// lives in one fixed static device array instead of a
 // caller-provided workspace.
 // ---------------------------------------------------------------------------
 namespace bitsmoe {

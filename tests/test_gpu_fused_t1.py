@@ -68,11 +68,12 @@ def test_fused_t1_repeated_calls_interleaved_with_batches():
             assert rel_err(out[f"Y_sum_{proj}"].cpu().numpy(), ref[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-5
         if it % 7 == 3:
             lay.forward(case.x[:5].contiguous(), case.ids[:5].contiguous(), case.gate_w[:5].contiguous())
-    # the same call twice gives bit-identical results (ordered routed sum)
+    # the same call twice agrees to fp32 rounding: the routed sum is accumulated
+    # with atomic adds, whose order may differ between runs
     a = _one(case, 3)
     b = _one(case, 3)
     for proj in ("gate", "up"):
-        assert torch.equal(a[f"Y_sum_{proj}"], b[f"Y_sum_{proj}"])
+        assert rel_err(a[f"Y_sum_{proj}"].cpu().numpy(), b[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-6
 
 
 def test_fused_t1_bad_expert_id():
