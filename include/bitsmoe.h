@@ -36,20 +36,20 @@
  *   - fp16 values are passed as uint16_t bit patterns; fp32 as float.
  *   - All arrays are dense, row-major, with the shapes written beside them.
  *
- * Packed format v1 (the blob written by bitsmoe_pack; little-endian).  Blob =
+ * Packed format v2 (the blob written by bitsmoe_pack; little-endian).  Blob =
  * header (64 B) | directory (E x 64 B) | expert 0 | expert 1 | ... ;
  * d_pad = roundup(d_out, 32).
- *   header: u32 magic "BMOE" | u32 version 1 | u32 d_out | u32 d_pad | u32 E |
+ *   header: u32 magic "BMOE" | u32 version 2 | u32 d_out | u32 d_pad | u32 E |
  *           u32 r | u64 total bytes | u64 64 | u64 64+64E | 16 zero bytes.
  *   directory entry e: u64 base (byte offset of expert e) | u64 bytes |
  *           u32 group offset from base [7] | u16 count [8] | u32 0;
  *           groups and counts in width order 16,8,6,4,3,2,1 (count[7] = width 0).
  *   group b in {1,2,3,4,6,8}, n members in ascending k, np = roundup(n,32):
  *           u16 idx[np] | u16 fp16 scale[np] | f32 amp[np] |
- *           u32 planes[d_pad/32][b][np/32][32]: bit m of word [t][j][w][i'] is
- *           bit j of q for member 32w+m at row 32t+i' (32-row tiles; a warp
- *           reads one plane word of 32 rows as 128 contiguous bytes, and a run
- *           of row tiles of one group is one contiguous block).
+ *           u32 planes[b][np/32][d_pad]: bit m of word [j][w][i] is bit j of
+ *           q for member 32w+m at row i (rows fastest: a warp reads one plane
+ *           word of 32 rows as 128 contiguous bytes, and consecutive plane
+ *           words of one group, all rows, are one contiguous block).
  *   group 16, np = roundup(n,8): u16 idx[np] | f32 amp[np] | u16 w16[np][d_pad].
  *   Every padding byte (members >= n, rows >= d_out) is zero.
  */

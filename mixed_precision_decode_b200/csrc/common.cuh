@@ -1,6 +1,6 @@
 // common.cuh -- internal definitions shared by the library's CUDA sources.
 //
-// The packed format (v1) and the quantiser are specified in include/bitsmoe.h;
+// The packed format (v2) and the quantiser are specified in include/bitsmoe.h;
 // this file is the library's own reading of that specification.
 #pragma once
 
@@ -37,7 +37,7 @@ __host__ __device__ inline bool width_ok(int b) {
 __host__ __device__ constexpr uint64_t roundup(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
 
 constexpr uint32_t kMagic = 0x454F4D42u;  // "BMOE"
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 constexpr uint64_t kHeaderBytes = 64;
 constexpr uint64_t kDirEntryBytes = 64;
 
@@ -53,10 +53,10 @@ __host__ __device__ inline uint64_t group_bytes(int b, uint64_t n, uint64_t d_pa
     return 8 * np + 4 * (uint64_t)b * (np / 32) * d_pad;
 }
 
-// Word index of plane word [tile i/32][plane j][word w][row i%32] inside a
-// group's planes (32-row tiles; W = words per plane, b = planes).
-__host__ __device__ inline uint64_t plane_word(uint32_t j, uint32_t w, uint32_t W, int b, uint32_t i) {
-    return ((((uint64_t)(i >> 5) * (uint64_t)b + j) * W + w) << 5) + (i & 31u);
+// Word index of plane word [plane j][word w][row i] inside a group's planes
+// (rows fastest; W = words per plane, d_pad = padded rows).
+__host__ __device__ inline uint64_t plane_word(uint32_t j, uint32_t w, uint32_t W, uint32_t d_pad, uint32_t i) {
+    return ((uint64_t)j * W + w) * d_pad + i;
 }
 
 // Directory entry of one expert, decoded.
@@ -89,7 +89,7 @@ struct QGroup {
     const uint16_t* idx;
     const uint16_t* scale;
     const float* amp;
-    const uint32_t* planes;  // [d_pad/32][b][W][32]
+    const uint32_t* planes;  // [b][W][d_pad]
     uint32_t n, np, W;
 };
 __device__ inline QGroup qgroup(const uint8_t* blob, const DirEntry& d, int g) {

@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     float2* s_tab = reinterpret_cast<float2*>(smem + P.sm_tab + (tab_s - tab_raw));
     float* s_red = reinterpret_cast<float*>(s_tab);  // reused after the last chunk: [warp][32][kMtTok]
 
-    // ---- stage the expert's metadata and this CTA's tiles of every group ----
-    if (tid == 0) {
+    // ---- stage the expert's metadata and this CTA's rows of every plane word ----
+    if (warp == 0) {
+      if (lane == 0) {
         const DirEntry d = read_dir(P.blob, e);
         uint32_t so = 0, mo = 0, co = 0;
         for (int g = 0; g < kNumGroups; g++) {
@@ -150,17 +151,28 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
         for (int g = 0; g < kNumGroups; g++) {
             if (s_ex.n[g] == 0) continue;
             const int b = group_width(g);
-            const uint8_t* G = P.blob + s_ex.gbase[g];
-            mt_bulk(s_meta + s_ex.meta_off[g], G, (b == 16 ? 6u : 8u) * s_ex.np[g], &s_bar);
-            if (b != 16) {
-                const uint32_t tw = (uint32_t)b * s_ex.W[g] * 32;  // words of one tile of this group
-                mt_bulk(s_stage + s_ex.stage_off[g], G + 8ull * s_ex.np[g] + 4ull * tw * tile0, 4u * tw * ntl, &s_bar);
-            }
+            mt_bulk(s_meta + s_ex.meta_off[g], P.blob + s_ex.gbase[g], (b == 16 ? 6u : 8u) * s_ex.np[g], &s_bar);
         }
-        if (!mt_mbar_wait(&s_bar, 0)) {
-            s_fail = 1;
-            if (P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
-        }
+      }
+      __syncwarp();
+      // plane word q of group g: rows [32 tile0, 32 (tile0 + ntl)) are contiguous in the
+      // blob ([b][W][d_pad], rows fastest) and staged as [b][W][32 ntl]
+      const uint64_t d_pad = 32ull * P.n_tiles;
+      int g = 1, qg = 0;  // group of plane word q, and its first word
+      for (int q = lane;; q += 32) {
+          while (g < kNumGroups && q >= qg + group_width(g) * (int)s_ex.W[g]) {
+              qg += group_width(g) * (int)s_ex.W[g];
+              g++;
+          }
+          if (g >= kNumGroups) break;
+          const uint8_t* planes = P.blob + s_ex.gbase[g] + 8ull * s_ex.np[g];
+          mt_bulk(s_stage + s_ex.stage_off[g] + (uint32_t)(q - qg) * 32u * ntl,
+                  planes + 4ull * ((uint64_t)(q - qg) * d_pad + 32ull * tile0), 128u * ntl, &s_bar);
+      }
+      if (lane == 0 && !mt_mbar_wait(&s_bar, 0)) {
+          s_fail = 1;
+          if (P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
+      }
     }
     __syncthreads();
     if (s_fail) return;
@@ -245,7 +257,7 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                 if (!tile_ok) continue;
                 for (int q = part; q < b * cw; q += wpt) {
                     const int j = q / cw, wi = q - j * cw;
-                    const uint32_t word = stg[(((uint32_t)my_tile * b + j) * W + w0 + wi) * 32 + lane];
+                    const uint32_t word = stg[(((uint32_t)j * W + w0 + wi) * ntl + my_tile) * 32 + lane];
                     // entry offsets (nibble x 8 bytes): even nibbles in the bytes of lo, odd in hi
                     const uint32_t lo = (word << 3) & 0x78787878u, hi = (word >> 1) & 0x78787878u;
                     const uint32_t base = tab_s + 2048u * (uint32_t)wi;  // (wi, pair 0); pair 1 at +1024

@@ -211,8 +211,7 @@ __device__ __forceinline__ void decode_pw(const UnitInfo& U, int q, int& g, int&
 // One work item of a CTA: a plane word (all rows of one bit plane of 32
 // members) or an octet of fp16 members (all rows).
 struct Item {
-    const uint8_t* ptr;  // plane word: its 32 words in tile 0; octet: member row 8f
-    uint32_t stride;     // plane word: bytes between the word's tiles
+    const uint8_t* ptr;  // plane word: its d_pad words (one per row); octet: member row 8f
     int16_t nf;          // octet: fp16 members in it (1..8); plane word: 0
     int16_t slot;        // member-word slot (plane word) or octet slot
     int16_t w;           // octet: f
@@ -227,11 +226,10 @@ struct MemberWord {
     int16_t zp;      // 1 when this CTA evaluates the word's plane 0 and so owns its zero-point share
     int16_t seg;
 };
-// Consecutive plane-word items of one group: contiguous in every 32-row tile,
-// so one bulk copy per tile stages all of them.
+// Consecutive plane-word items of one group: contiguous in the blob (planes
+// are [b][W][d_pad], rows fastest), so one bulk copy stages all of them.
 struct Run {
-    const uint8_t* ptr;  // the first item's words in tile 0
-    uint32_t stride;     // bytes between tiles
+    const uint8_t* ptr;  // the first item's words
     int a, len;          // first item slot, items
 };
 // Items of one unit inside a CTA's share: plane words [i0, ip), fp16 octets [ip, i1).
@@ -272,7 +270,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     uint16_t* s_x = reinterpret_cast<uint16_t*>(smem + P.sm_x);
     uint8_t* s_dir = smem + P.sm_dir;  // [projection][expert] directory entries
     uint8_t* s_phi = smem + P.sm_phi;
-    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);  // [tile][item slot][32]
+    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);  // [item slot][d_pad]
     uint8_t* s_mwd = smem + P.sm_mw;    // [member word]: idx u16[32] | scale u16[32] | amp f32[32]
     uint8_t* s_f16d = smem + P.sm_f16;  // [octet]: idx u16[8] | amp f32[8]
     float* s_c16 = reinterpret_cast<float*>(smem + P.sm_c16);  // [octet][8]
@@ -355,15 +353,13 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             it.u = (int16_t)my_u;
             if (l < U.pw) {
                 decode_pw(U, l, g, jb, w);
-                const uint32_t b = (uint32_t)group_width(g), W = U.np[g] / 32;
-                it.ptr = blob + U.gbase[g] + 8ull * U.np[g] + 128ull * ((uint64_t)jb * W + (uint64_t)w);
-                it.stride = 128u * b * W;
+                const uint32_t W = U.np[g] / 32;
+                it.ptr = blob + U.gbase[g] + 8ull * U.np[g] + 4ull * P.d_pad * ((uint64_t)jb * W + (uint64_t)w);
                 it.nf = 0;
                 key = (my_u << 24) | (g << 16) | w;
             } else {
                 const int f = l - U.pw;
                 it.ptr = blob + U.gbase[0] + 6ull * U.np[0] + 2ull * kF16Item * (uint64_t)f * (uint64_t)P.d_pad;
-                it.stride = 0;
                 it.nf = (int16_t)min(kF16Item, U.n16 - kF16Item * f);
                 it.w = (int16_t)f;
             }
@@ -421,19 +417,17 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             S.ip = octs ? __ffs(octs) - 1 : i1;
             s_seg[seg] = S;
         }
-        // runs of plane words: consecutive items whose words are contiguous in every tile
+        // runs of plane words: consecutive items whose words follow each other in the blob
         const uint64_t my_ptr = (uint64_t)it.ptr;
         const uint64_t prev_ptr = __shfl_up_sync(0xffffffffu, my_ptr, 1);
-        const uint32_t prev_stride = __shfl_up_sync(0xffffffffu, it.stride, 1);
         const int prev_plane = __shfl_up_sync(0xffffffffu, (int)plane, 1);
-        const bool cont = plane && lane > 0 && prev_plane && prev_stride == it.stride && my_ptr == prev_ptr + 128u;
+        const bool cont = plane && lane > 0 && prev_plane && my_ptr == prev_ptr + 4ull * P.d_pad;
         const unsigned bcont = __ballot_sync(0xffffffffu, cont), bplane = __ballot_sync(0xffffffffu, plane);
         const unsigned brun = bplane & ~bcont;
         if ((brun >> lane) & 1u) {
             const unsigned stop = ~bcont & (lane == 31 ? 0u : ~((2u << lane) - 1u));  // first later item not continuing
             Run R;
             R.ptr = it.ptr;
-            R.stride = it.stride;
             R.a = lane;
             R.len = (stop ? __ffs(stop) - 1 : 32) - lane;
             s_run[__popc(brun & lt)] = R;
@@ -443,7 +437,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             s_nmw = __popc(bm);
             s_nseg = __popc(bs);
             s_nrun = __popc(brun);
-            s_stage_bytes = 128u * (uint32_t)__popc(bplane) * (uint32_t)P.n_rb + 256u * __popc(bm) + 48u * __popc(bf);
+            s_stage_bytes = 4u * (uint32_t)P.d_pad * (uint32_t)__popc(bplane) + 256u * __popc(bm) + 48u * __popc(bf);
             s_bad = bad;
         }
     }
@@ -474,22 +468,18 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         }
     }
 
-    // ---- staging by the staging warp (bulk copies on one mbarrier): plane-word runs
-    // into [tile][item slot], one copy per run and tile; then each member word's idx,
-    // scale and amp, and each octet's idx and amp ----
+    // ---- staging by the staging warp (bulk copies on one mbarrier): each run of plane
+    // words in one copy into [item slot][d_pad]; then each member word's idx, scale
+    // and amp, and each octet's idx and amp ----
     if (!row_warp) {
         const int st = threadIdx.x - nrw * 32, nst = kStageWarps * 32;
         const uint64_t stream = policy_evict_first();
         uint64_t* bar = &s_bar[kPhiBars + 1];
         if (st == 0) mbar_expect_tx(bar, s_stage_bytes);
         __syncwarp();
-        const uint32_t tstride = 128u * (uint32_t)P.items_max;  // bytes between tiles in s_planes
-        const int nr = s_nrun;
-        for (int pr = st; pr < nr * P.n_rb; pr += nst) {
-            const int r = pr / P.n_rb, t = pr - r * P.n_rb;
+        for (int r = st; r < s_nrun; r += nst) {
             const Run R = s_run[r];
-            bulk_g2s(reinterpret_cast<uint8_t*>(s_planes) + (size_t)t * tstride + 128u * R.a,
-                     R.ptr + (uint64_t)t * R.stride, 128u * (uint32_t)R.len, bar, stream);
+            bulk_g2s(s_planes + (size_t)R.a * P.d_pad, R.ptr, 4u * (uint32_t)P.d_pad * (uint32_t)R.len, bar, stream);
         }
         for (int m = st; m < nmw; m += nst) {
             const MemberWord& M = s_mw[m];
@@ -618,12 +608,12 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         // this CTA's zero-point share of the unit (member words in slot order)
         const float zps = warp_sum(lane < nmw && s_mw[lane].seg == s ? s_zpmw[lane] : 0.0f);
         for (int t = warp; t < P.n_rb; t += nwarps) {
-            const uint32_t* pl = s_planes + (size_t)t * P.items_max * kRB + lane;  // [tile][item slot][32]
+            const uint32_t* pl = s_planes + t * kRB + lane;  // [item slot][d_pad]
             float acc = 0.0f;
 #pragma unroll 2
             for (int i = S.i0; i < S.ip; i++) {
                 const uint2 d = s_desc[i];
-                const uint32_t word = pl[i * kRB];
+                const uint32_t word = pl[i * P.d_pad];
                 // entry offsets (nibble x 4 bytes): even nibbles in the bytes of lo, odd in hi;
                 // table n of this word is at d.x + 64 n, entry e at + 4 e
                 const uint32_t lo = (word << 2) & 0x3C3C3C3Cu, hi = (word >> 2) & 0x3C3C3C3Cu;

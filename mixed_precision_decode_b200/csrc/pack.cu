@@ -165,7 +165,7 @@ __device__ void pack_word(const float* __restrict__ comps_e, const uint16_t* idx
             for (int j = 0; j < B; j++) word[j] |= ((q >> j) & 1u) << m;
         }
 #pragma unroll
-        for (int j = 0; j < B; j++) planes[plane_word(j, w, W, B, i)] = word[j];
+        for (int j = 0; j < B; j++) planes[plane_word(j, w, W, d_pad, i)] = word[j];
     }
 }
 
@@ -228,7 +228,7 @@ __global__ void k_unpack(const uint8_t* __restrict__ blob, uint16_t* __restrict_
     const uint32_t valid = min(32u, q.n - 32 * item.w);
     for (uint32_t i = blockIdx.z * blockDim.x + threadIdx.x; i < (uint32_t)d_out; i += gridDim.z * blockDim.x) {
         uint32_t word[8];
-        for (int j = 0; j < b; j++) word[j] = q.planes[plane_word(j, item.w, q.W, b, i)];
+        for (int j = 0; j < b; j++) word[j] = q.planes[plane_word(j, item.w, q.W, d_pad, i)];
         for (uint32_t m = 0; m < valid; m++) {
             uint32_t v = 0;
             for (int j = 0; j < b; j++) v |= ((word[j] >> m) & 1u) << j;

@@ -11,7 +11,7 @@ from . import bitsmoe as B
 class PackedProjection:
     """One projection (gate or up) of a spectral MoE layer, packed on the GPU.
 
-    phi_t [r][d_in] fp16 (rows phi_k, kept unquantised), blob = the format-v1
+    phi_t [r][d_in] fp16 (rows phi_k, kept unquantised), blob = the format-v2
     bit-plane blob of the expert directions, plan = its host descriptor."""
 
     def __init__(self, plan: B.Plan, blob: torch.Tensor, phi_t: torch.Tensor):

@@ -156,7 +156,7 @@ def compute_scales(comps: np.ndarray, widths: np.ndarray) -> tuple[np.ndarray, i
 
 
 def pack(comps: np.ndarray, widths: np.ndarray, scales: np.ndarray, amps: np.ndarray) -> tuple[np.ndarray, int]:
-    """Pack into the format-v1 blob; returns (blob uint8, status)."""
+    """Pack into the format-v2 blob; returns (blob uint8, status)."""
     comps = _c(comps, np.float32)
     w = _c(widths, np.uint8)
     s = _c(scales, np.uint16)

@@ -105,7 +105,7 @@ double orc_f16_to_f64(uint16_t h) {
 static float orc_f16_to_f32(uint16_t h) { return (float)orc_f16_to_f64(h); }
 
 /* ------------------------------------------------------------------------- */
-/* Widths and the packed layout (format v1).                                 */
+/* Widths and the packed layout (format v2).                                 */
 /* ------------------------------------------------------------------------- */
 
 static int orc_width_ok(int b) {
@@ -126,10 +126,10 @@ static uint64_t orc_group_bytes(int b, uint64_t n, uint64_t d_pad) {
     return 2 * np + 2 * np + 4 * np + 4 * (uint64_t)b * (np / 32) * d_pad; /* idx, scale, amp, planes */
 }
 
-/* Byte offset of plane word [tile i/32][plane j][word w][row i%32] inside a
- * group's planes; W = words per plane. */
-static uint64_t orc_plane_off(uint64_t j, uint64_t w, uint64_t W, int b, uint64_t i) {
-    return 4 * ((((i / 32) * (uint64_t)b + j) * W + w) * 32 + i % 32);
+/* Byte offset of plane word [plane j][word w][row i] inside a group's planes
+ * (rows fastest); W = words per plane, d_pad = padded rows. */
+static uint64_t orc_plane_off(uint64_t j, uint64_t w, uint64_t W, uint64_t d_pad, uint64_t i) {
+    return 4 * ((j * W + w) * d_pad + i);
 }
 
 /* Count of each width for expert e: cnt[g] for groups g = 0..6 (widths
@@ -256,7 +256,7 @@ uint32_t orc_quantise(float p, int b, uint16_t sh, int32_t *st) {
 /* ------------------------------------------------------------------------- */
 
 /* Pack comps [E][r][d_out] (unit directions p_{e,k}), amps [E][r] and fp16
- * scales [E][r] into the format-v1 blob.  Every byte of the blob is written
+ * scales [E][r] into the format-v2 blob.  Every byte of the blob is written
  * (padding included).  Returns 0 or a negative error; data errors go to
  * *status as bits. */
 int orc_pack(int E, int r, int d_out, const uint8_t *widths, const float *comps,
@@ -273,7 +273,7 @@ int orc_pack(int E, int r, int d_out, const uint8_t *widths, const float *comps,
 
     /* header */
     put32(blob + 0, 0x454F4D42u); /* "BMOE" */
-    put32(blob + 4, 1u);
+    put32(blob + 4, 2u);
     put32(blob + 8, (uint32_t)d_out);
     put32(blob + 12, (uint32_t)d_pad);
     put32(blob + 16, (uint32_t)E);
@@ -337,7 +337,7 @@ int orc_pack(int E, int r, int d_out, const uint8_t *widths, const float *comps,
                             uint32_t q = orc_quantise(p[i], b, sh, &st);
                             for (int j = 0; j < b; j++) {
                                 if (!((q >> j) & 1u)) continue;
-                                uint8_t *word = planes + orc_plane_off((uint64_t)j, w, W, b, (uint64_t)i);
+                                uint8_t *word = planes + orc_plane_off((uint64_t)j, w, W, d_pad, (uint64_t)i);
                                 put32(word, get32(word) | (1u << bit));
                             }
                         }
@@ -364,7 +364,7 @@ int orc_pack(int E, int r, int d_out, const uint8_t *widths, const float *comps,
  * Returns 0 and fills the dims, or ORC_EFORMAT. */
 int orc_blob_parse(const uint8_t *blob, uint64_t bytes, int *E, int *r, int *d_out) {
     if (!blob || bytes < 64) return ORC_EFORMAT;
-    if (get32(blob) != 0x454F4D42u || get32(blob + 4) != 1u) return ORC_EFORMAT;
+    if (get32(blob) != 0x454F4D42u || get32(blob + 4) != 2u) return ORC_EFORMAT;
     uint64_t dout = get32(blob + 8), dpad = get32(blob + 12), ne = get32(blob + 16), rk = get32(blob + 20);
     if (!orc_dims_ok((int)ne, (int)rk, (int)dout) || dpad != orc_roundup(dout, 32)) return ORC_EFORMAT;
     uint64_t total = get64(blob + 24);
@@ -450,7 +450,7 @@ int orc_unpack(const uint8_t *blob, uint64_t bytes, uint16_t *q, uint8_t *widths
                         for (int i = 0; i < d_out; i++) {
                             uint32_t v = 0;
                             for (int j = 0; j < b; j++) {
-                                uint32_t word = get32(planes + orc_plane_off((uint64_t)j, m / 32, W, b, (uint64_t)i));
+                                uint32_t word = get32(planes + orc_plane_off((uint64_t)j, m / 32, W, d_pad, (uint64_t)i));
                                 v |= ((word >> (m % 32)) & 1u) << j;
                             }
                             q[ek * d_out + i] = (uint16_t)v;
@@ -564,7 +564,7 @@ int orc_expert_forward(const uint8_t *blob, uint64_t bytes, const double *Z, con
                                 uint64_t W = np / 32;
                                 uint32_t v = 0;
                                 for (int j = 0; j < b; j++) {
-                                    uint32_t word = get32(G + 8 * np + orc_plane_off((uint64_t)j, m / 32, W, b, (uint64_t)i));
+                                    uint32_t word = get32(G + 8 * np + orc_plane_off((uint64_t)j, m / 32, W, d_pad, (uint64_t)i));
                                     v |= ((word >> (m % 32)) & 1u) << j;
                                 }
                                 qv = (uint16_t)v;

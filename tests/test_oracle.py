@@ -110,6 +110,26 @@ def test_golden_unpack_and_dequant(orc):
         assert np.all(ae[~stored] == 0)
 
 
+def test_golden_rows_layout(orc):
+    """A second hand-derived blob, 40 rows and two planes: where each plane word sits."""
+    with open(os.path.join(GOLDEN, "layout_rows.json")) as f:
+        g = json.load(f)
+    comps, widths, amps = _golden_inputs(g)
+    scales, st = orc.compute_scales(comps, widths)
+    assert st == 0 and scales.tolist() == g["scales"]
+    blob, st = orc.pack(comps, widths, scales, amps)
+    assert st == 0
+    expect = np.zeros(g["total_bytes"], np.uint8)
+    for off, hexs in g["nonzero"].items():
+        b = bytes.fromhex(hexs.replace(" ", ""))
+        expect[int(off):int(off) + len(b)] = np.frombuffer(b, np.uint8)
+    assert blob.size == expect.size
+    diff = np.flatnonzero(blob != expect)
+    assert diff.size == 0, [(int(o), int(blob[o]), int(expect[o])) for o in diff[:16]]
+    q, _, _, _ = orc.unpack(blob)
+    assert q.tolist() == g["q"]
+
+
 def test_golden_forward_by_hand(orc):
     """Y for one token with a hand-chosen z, worked out from the golden dequantised values."""
     g = _golden()
@@ -257,7 +277,7 @@ def test_roundtrip_and_padding(orc, shape):
 
 
 def _plane_popcount(blob, E):
-    """Independent reader of the format-v1 directory: popcount over every plane word."""
+    """Independent reader of the format-v2 directory: popcount over every plane word."""
     blob = np.asarray(blob, np.uint8)
     d_pad = int(blob[12:16].view(np.uint32)[0])
     total = 0
