@@ -160,9 +160,12 @@ class Workload:
     def layer_of(self, s):
         return s % len(self.layers)
 
-    def step(self, s, stream=None):
+    def step(self, s, stream=None, next_s=None):
+        """Step s; with next_s, as a decode loop that runs step next_s after it
+        (its layer's Phi^T is prefetched while this step evaluates experts)."""
         l = self.layer_of(s)
-        self.layers[l].forward(self.x[s], self.ids[s], self.gw[s], out=self.out[l], stream=stream)
+        nxt = None if next_s is None else self.layers[self.layer_of(next_s)]
+        self.layers[l].forward(self.x[s], self.ids[s], self.gw[s], out=self.out[l], stream=stream, next_layer=nxt)
 
     def blob_bytes_total(self):
         return sum(L.gate.blob.numel() + L.up.blob.numel() + 2 * L.gate.phi_t.numel() * 2 for L in self.layers) // 2 * 2
@@ -362,36 +365,54 @@ def run_ours(args, dist):
     bys = [algorithmic_bytes(cfg, wl.counts[wl.layer_of(s)], wl.ids[s].cpu().numpy(), T) for s in range(G)]
     alg = {k: float(np.mean([b[k] for b in bys])) for k in bys[0]}
 
-    # warm-up (eager), then capture G steps into a graph (and the remainder)
-    for s in range(W):
-        wl.step(s % G)
-    torch.cuda.synchronize()
-    graphs = []
-    for n in ([G] * (K // G)) + ([K % G] if K % G else []):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=torch.cuda.Stream()):
-            for s in range(n):
-                wl.step(s)
-        graphs.append(g)
-    for g in graphs[:2]:
-        g.replay()
-    torch.cuda.synchronize()
+    # warm-up (eager), then capture G steps into a graph (and the remainder).  The
+    # steps run as a decode loop: each call names the layer that runs next (it
+    # wraps at the end of a graph, where the next replay starts again at step 0).
+    def capture(chained):
+        for s in range(W):
+            wl.step(s % G, next_s=((s + 1) % G) if chained else None)
+        torch.cuda.synchronize()
+        gs = []
+        for n in ([G] * (K // G)) + ([K % G] if K % G else []):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=torch.cuda.Stream()):
+                for s in range(n):
+                    wl.step(s, next_s=((s + 1) % n) if chained else None)
+            gs.append(g)
+        for g in gs[:2]:
+            g.replay()
+        torch.cuda.synchronize()
+        return gs
 
-    clocks = ClockSampler(torch.cuda.current_device())
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    torch.cuda.synchronize()
-    with clocks:
-        torch.cuda.nvtx.range_push("timed")
+    def timed(gs, clocks=None, nvtx=False):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        if clocks:
+            clocks.__enter__()
+        if nvtx:
+            torch.cuda.nvtx.range_push("timed")
         ev0.record(stream)
-        for g in graphs:
+        for g in gs:
             g.replay()
         ev1.record(stream)
         torch.cuda.synchronize()
-        torch.cuda.nvtx.range_pop()
-    dist.barrier()
-    ms = dist.max(ev0.elapsed_time(ev1))
+        if nvtx:
+            torch.cuda.nvtx.range_pop()
+        if clocks:
+            clocks.__exit__(None, None, None)
+        dist.barrier()
+        return dist.max(ev0.elapsed_time(ev1))
+
+    # the same loop as a chained decode loop (next layer's Phi^T prefetched into L2), reported beside
+    graphs = capture(True)
+    ms_chained = timed(graphs)
+    del graphs
+    graphs = capture(False)
+    clocks = ClockSampler(torch.cuda.current_device())
+    ms = timed(graphs, clocks, nvtx=True)
     value, step_s = weak_scaling_throughput(dist.world, K, T, ms)
+    value_ch, step_ch = weak_scaling_throughput(dist.world, K, T, ms_chained)
 
     peak, peak_kind = load_peak()
     achieved = alg["total"] / step_s / 1e9
@@ -416,6 +437,10 @@ def run_ours(args, dist):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "chained": {"value": value_ch, "ms_per_step": step_ch * 1e3,
+                    "roofline_frac": alg["total"] / step_ch / 1e9 / peak,
+                    "how": "the same graph-replayed loop through bitsmoe_layer_forward_chained: each call prefetches "
+                           "the next step's layer Phi^T into L2 while it evaluates experts"},
     }
     if want_cpu:
         samp = OracleSample(wl, [0 if args.layers == 1 else s for s in range(0, 4 * args.layers, args.layers)][:4])

@@ -197,6 +197,26 @@ int bitsmoe_layer_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up
                           const int32_t *topk_ids, const float *gate_w, int32_t T, void *workspace,
                           uint64_t workspace_bytes, int32_t *status, void *stream);
 
+/* bitsmoe_layer_forward for a decode loop that knows the layer it runs next.
+ * The BitsMoE pages have no counterpart to this call: at one token the shared
+ * projections' Phi^T are most of the bytes a layer reads, and they are
+ * weights, known before the next layer's input exists.  So while this call
+ * evaluates its experts (when HBM would otherwise be idle) the fused
+ * single-token path prefetches next_phi_t_gate and next_phi_t_up -- the next
+ * layer's Phi^T, dev [r][d_in] fp16 each, the same shape as this layer's --
+ * into L2, and the next call reads them from there.  The bytes still come
+ * from HBM once per layer; only their time moves.  Other paths (T > 1, or
+ * shapes the fused path does not take) ignore the two pointers.
+ *   Arguments as in bitsmoe_layer_forward, plus next_phi_t_gate / next_phi_t_up:
+ *   both NULL (no prefetch, the same as bitsmoe_layer_forward) or both
+ *   16-byte aligned device pointers; nothing is written through them.
+ * Errors: those of bitsmoe_layer_forward; EINVAL when only one is NULL or one
+ * is misaligned. */
+int bitsmoe_layer_forward_chained(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,
+                                  const int32_t *topk_ids, const float *gate_w, int32_t T, void *workspace,
+                                  uint64_t workspace_bytes, const uint16_t *next_phi_t_gate,
+                                  const uint16_t *next_phi_t_up, int32_t *status, void *stream);
+
 /* Single-token layer forward (T = 1) that allocates nothing: the same fused
  * kernel as bitsmoe_layer_forward, with its scratch taken from one fixed 1 MiB
  * array that the library keeps in device memory (every GPU that loads the

@@ -24,7 +24,7 @@ EXPORTS = (
     "bitsmoe_plan_header_bytes", "bitsmoe_plan_get_dims", "bitsmoe_plan_write_header", "bitsmoe_compute_scales",
     "bitsmoe_pack", "bitsmoe_unpack_q", "bitsmoe_shared_proj", "bitsmoe_expert_workspace_bytes",
     "bitsmoe_expert_forward", "bitsmoe_layer_workspace_bytes", "bitsmoe_layer_launches", "bitsmoe_layer_forward",
-    "bitsmoe_layer_forward_t1_noalloc", "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
+    "bitsmoe_layer_forward_chained", "bitsmoe_layer_forward_t1_noalloc", "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
 )
 
 
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             "bitsmoe_layer_launches": ([vp, vp, i32], ctypes.c_int),
             "bitsmoe_layer_forward": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, i32, vp, u64,
                                        vp, vp], ctypes.c_int),
+            "bitsmoe_layer_forward_chained": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, i32, vp,
+                                               u64, vp, vp, vp, vp], ctypes.c_int),
             "bitsmoe_layer_forward_t1_noalloc": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, vp,
                                                   vp], ctypes.c_int),
             "bitsmoe_read_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
@@ -215,6 +217,15 @@ def layer_forward(gate: ProjIO, up: ProjIO, X, topk_ids, gate_w, T: int, workspa
     _check(lib().bitsmoe_layer_forward(ctypes.byref(gate), ctypes.byref(up), _ptr(X), _ptr(topk_ids), _ptr(gate_w),
                                        T, _ptr(workspace), workspace_bytes, _ptr(status), _stream(stream)),
            "layer_forward")
+
+
+def layer_forward_chained(gate: ProjIO, up: ProjIO, X, topk_ids, gate_w, T: int, workspace, workspace_bytes: int,
+                          next_phi_t_gate, next_phi_t_up, status=None, stream=None):
+    _check(lib().bitsmoe_layer_forward_chained(ctypes.byref(gate), ctypes.byref(up), _ptr(X), _ptr(topk_ids),
+                                               _ptr(gate_w), T, _ptr(workspace), workspace_bytes,
+                                               _ptr(next_phi_t_gate), _ptr(next_phi_t_up), _ptr(status),
+                                               _stream(stream)),
+           "layer_forward_chained")
 
 
 def layer_forward_t1_noalloc(gate: ProjIO, up: ProjIO, X, topk_ids, gate_w, status=None, stream=None):

@@ -203,7 +203,8 @@ static uint64_t layer_ws(const bitsmoe_plan* g, const bitsmoe_plan* u, int T, co
 }
 
 int layer_forward_fused_t1(const bitsmoe_proj_io* io[2], const uint16_t* X, const int32_t* ids, const float* gw,
-                           void* workspace, uint64_t workspace_bytes, int32_t* status, cudaStream_t s, bool* used);
+                           void* workspace, uint64_t workspace_bytes, const uint16_t* const* next_phi, int32_t* status,
+                           cudaStream_t s, bool* used);
 uint64_t layer_fused_t1_workspace(const bitsmoe_plan* g, const bitsmoe_plan* u);
 uint64_t layer_fused_t1_reserved(const bitsmoe_plan* g, const bitsmoe_plan* u);
 }  // namespace bitsmoe
@@ -224,9 +225,9 @@ BITSMOE_API int bitsmoe_layer_launches(const bitsmoe_plan* gate, const bitsmoe_p
     return 7;  // route, then per projection: shared projection, experts, combine
 }
 
-BITSMOE_API int bitsmoe_layer_forward(const bitsmoe_proj_io* gate, const bitsmoe_proj_io* up, const uint16_t* X,
-                                      const int32_t* topk_ids, const float* gate_w, int32_t T, void* workspace,
-                                      uint64_t workspace_bytes, int32_t* status, void* stream) {
+static int layer_forward_impl(const bitsmoe_proj_io* gate, const bitsmoe_proj_io* up, const uint16_t* X,
+                              const int32_t* topk_ids, const float* gate_w, int32_t T, void* workspace,
+                              uint64_t workspace_bytes, const uint16_t* const* next_phi, int32_t* status, void* stream) {
     if (!gate || !up || T < 0 || !gate->plan || !up->plan) return BITSMOE_EINVAL;
     const bitsmoe_proj_io* io[2] = {gate, up};
     const bitsmoe_plan *pg = gate->plan, *pu = up->plan;
@@ -245,7 +246,7 @@ BITSMOE_API int bitsmoe_layer_forward(const bitsmoe_proj_io* gate, const bitsmoe
     cudaStream_t s = (cudaStream_t)stream;
     if (T == 1) {
         bool used = false;
-        int rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, workspace, workspace_bytes, status, s, &used);
+        int rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, workspace, workspace_bytes, next_phi, status, s, &used);
         if (rc || used) return rc;
     }
     LayerWS L;
@@ -262,4 +263,22 @@ BITSMOE_API int bitsmoe_layer_forward(const bitsmoe_proj_io* gate, const bitsmoe
         if (rc) return rc;
     }
     return BITSMOE_OK;
+}
+
+BITSMOE_API int bitsmoe_layer_forward(const bitsmoe_proj_io* gate, const bitsmoe_proj_io* up, const uint16_t* X,
+                                      const int32_t* topk_ids, const float* gate_w, int32_t T, void* workspace,
+                                      uint64_t workspace_bytes, int32_t* status, void* stream) {
+    return layer_forward_impl(gate, up, X, topk_ids, gate_w, T, workspace, workspace_bytes, nullptr, status, stream);
+}
+
+BITSMOE_API int bitsmoe_layer_forward_chained(const bitsmoe_proj_io* gate, const bitsmoe_proj_io* up,
+                                              const uint16_t* X, const int32_t* topk_ids, const float* gate_w,
+                                              int32_t T, void* workspace, uint64_t workspace_bytes,
+                                              const uint16_t* next_phi_t_gate, const uint16_t* next_phi_t_up,
+                                              int32_t* status, void* stream) {
+    if ((next_phi_t_gate == nullptr) != (next_phi_t_up == nullptr)) return BITSMOE_EINVAL;
+    if ((uintptr_t)next_phi_t_gate % 16 || (uintptr_t)next_phi_t_up % 16) return BITSMOE_EINVAL;
+    const uint16_t* next[2] = {next_phi_t_gate, next_phi_t_up};
+    return layer_forward_impl(gate, up, X, topk_ids, gate_w, T, workspace, workspace_bytes,
+                              next_phi_t_gate ? next : nullptr, status, stream);
 }

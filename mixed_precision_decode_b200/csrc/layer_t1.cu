@@ -53,6 +53,7 @@ struct T1Proj {
 
 struct T1Params {
     T1Proj proj[2];
+    const uint16_t* next_phi[2];  // the next layer's Phi^T (both projections) to prefetch into L2, or null
     const uint16_t* x;
     const int32_t* ids;
     const float* gw;
@@ -120,6 +121,9 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
     asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
@@ -559,6 +563,15 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
         return;
     }
+    // Every CTA has read its Phi: HBM is free while the experts are evaluated, so
+    // pull this CTA's rows of the next layer's Phi into L2 for the next call.
+    if (tid == 0 && P.next_phi[0] && P.next_phi[1])
+        for (int rr = row0; rr < row1;) {
+            const int p = rr / P.r, k = rr - p * P.r;
+            const int n = min(row1 - rr, P.r - k);
+            bulk_prefetch_l2(P.next_phi[p] + (size_t)k * P.d_in, (uint32_t)n * row_bytes);
+            rr += n;
+        }
 
     // ---- c_k = a_k s_k z_k, the tables and the zero-point share: a warp per member word ----
     for (int m = warp; m < nmw; m += nwarps) {
@@ -765,7 +778,8 @@ uint64_t layer_fused_t1_reserved(const bitsmoe_plan* g, const bitsmoe_plan* u) {
 }
 
 int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const int32_t* ids, const float* gw,
-                           void* workspace, uint64_t workspace_bytes, int32_t* status, cudaStream_t s, bool* used) {
+                           void* workspace, uint64_t workspace_bytes, const uint16_t* const* next_phi, int32_t* status,
+                           cudaStream_t s, bool* used) {
     *used = false;
     T1Layout L = t1_layout(io[0]->plan, io[1]->plan);
     if (!L.ok || workspace_bytes < L.ws_reserved + L.ws_bytes) return BITSMOE_OK;
@@ -777,6 +791,8 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
         P.proj[j].Ye = io[j]->Y_experts;
         P.proj[j].Ysum = io[j]->Y_sum;
     }
+    P.next_phi[0] = next_phi ? next_phi[0] : nullptr;
+    P.next_phi[1] = next_phi ? next_phi[1] : nullptr;
     P.x = X;
     P.ids = ids;
     P.gw = gw;
@@ -868,7 +884,7 @@ BITSMOE_API int bitsmoe_layer_forward_t1_noalloc(const bitsmoe_proj_io* gate, co
     cudaError_t e = cudaMemsetAsync(scratch, 0, head, s);
     if (e != cudaSuccess) return set_cuda_error(e);
     bool used = false;
-    rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, scratch, head + rest, status, s, &used);
+    rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, scratch, head + rest, nullptr, status, s, &used);
     if (rc) return rc;
     return used ? BITSMOE_OK : BITSMOE_ESIZE;
 }

@@ -66,9 +66,11 @@ class SpectralMoELayer:
 
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, gate_w: torch.Tensor, out: dict | None = None,
                 want_experts: bool = False, want_z: bool = False, status: torch.Tensor | None = None,
-                stream=None) -> dict:
+                stream=None, next_layer: "SpectralMoELayer | None" = None) -> dict:
         """x [T][d_in] fp16, topk_ids [T][top_k] int32, gate_w [T][top_k] f32 (all on the GPU).
-        Returns Y_sum_gate / Y_sum_up [T][d_out] f32 (and Y_experts_* / Z_* on request)."""
+        Returns Y_sum_gate / Y_sum_up [T][d_out] f32 (and Y_experts_* / Z_* on request).
+        next_layer: the layer a decode loop runs next; its Phi^T are prefetched into
+        L2 while this call evaluates its experts (single-token path)."""
         T = x.shape[0]
         dev = x.device
         if out is None:
@@ -84,5 +86,9 @@ class SpectralMoELayer:
             ios.append(B.proj_io(p.plan, p.blob, p.phi_t, out[f"Y_sum_{name}"], out.get(f"Z_{name}"),
                                  out.get(f"Y_experts_{name}")))
         ws = self.workspace(T)
-        B.layer_forward(ios[0], ios[1], x, topk_ids, gate_w, T, ws, ws.numel(), status, stream)
+        if next_layer is None:
+            B.layer_forward(ios[0], ios[1], x, topk_ids, gate_w, T, ws, ws.numel(), status, stream)
+        else:
+            B.layer_forward_chained(ios[0], ios[1], x, topk_ids, gate_w, T, ws, ws.numel(), next_layer.gate.phi_t,
+                                    next_layer.up.phi_t, status, stream)
         return out

@@ -116,3 +116,13 @@ def test_argument_checks_before_any_launch(B):
     assert L.bitsmoe_layer_forward(ctypes.byref(io), ctypes.byref(io), 256, 256, 256, 2, 256, nl - 1, None,
                                    None) == B.ESIZE
     assert B.strerror(B.EWIDTH).startswith("width")
+
+
+def test_chained_call_rejects_one_next_pointer(B):
+    """The next-layer pointers come in pairs and are 16-byte aligned; the checks run
+    before any device work."""
+    L = B.lib()
+    rc = L.bitsmoe_layer_forward_chained(None, None, None, None, None, 1, None, 0, 256, None, None, None)
+    assert rc == B.EINVAL
+    rc = L.bitsmoe_layer_forward_chained(None, None, None, None, None, 1, None, 0, 256, 264, None, None)
+    assert rc == B.EINVAL

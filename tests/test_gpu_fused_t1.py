@@ -69,11 +69,13 @@ def test_fused_t1_repeated_calls_interleaved_with_batches():
         if it % 7 == 3:
             lay.forward(case.x[:5].contiguous(), case.ids[:5].contiguous(), case.gate_w[:5].contiguous())
     # the same call twice agrees to fp32 rounding: the routed sum is accumulated
-    # with atomic adds, whose order may differ between runs
+    # with atomic adds, whose order may differ between runs.  Each element sums
+    # ~80 partials (8 slots x ~10 CTAs); fp32 summation in any order is within
+    # (n-1) * 2^-24 * sum|partials|, about 1e-5 of the vector's largest entry here.
     a = _one(case, 3)
     b = _one(case, 3)
     for proj in ("gate", "up"):
-        assert rel_err(a[f"Y_sum_{proj}"].cpu().numpy(), b[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-6
+        assert rel_err(a[f"Y_sum_{proj}"].cpu().numpy(), b[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-5
 
 
 def test_fused_t1_bad_expert_id():
@@ -111,3 +113,16 @@ def test_fused_t1_in_cuda_graph():
     for o in outs:
         for proj in ("gate", "up"):
             assert rel_err(o[f"Y_sum_{proj}"].cpu().numpy(), ref[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-5
+
+
+def test_chained_call_prefetch_changes_nothing(orc):
+    """A decode loop that names the next layer (its Phi^T is prefetched into L2)
+    gets the same outputs as the plain call, at one token and at several."""
+    case = get_case("qwen_t1")
+    lay = case.layer
+    for T in (1, 3):
+        x, ids, gw = case.x[:T].contiguous(), case.ids[:T].contiguous(), case.gate_w[:T].contiguous()
+        a = lay.forward(x, ids, gw, want_experts=True)
+        b = lay.forward(x, ids, gw, want_experts=True, next_layer=lay)
+        for k in a:
+            assert rel_err(a[k].cpu().numpy(), b[k].cpu().numpy()) <= 1e-6, (T, k)
