@@ -122,6 +122,14 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+// Named barrier `ID` over n threads (whole warps).  The callers come out of code
+// whose trip counts differ between lanes, so the warp is reconverged first:
+// bar.sync wants all 32 lanes to execute it together.
+template <int ID>
+__device__ __forceinline__ void named_barrier(int n) {
+    __syncwarp();
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(n) : "memory");
+}
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
@@ -236,6 +244,13 @@ struct Run {
     const uint8_t* ptr;  // the first item's words
     int a, len;          // first item slot, items
 };
+// Consecutive member-word slots of one group with consecutive words: their idx,
+// scale and amp are each one contiguous block in the blob and in shared memory.
+struct MetaRun {
+    const uint8_t* meta;  // the group's metadata
+    uint32_t np;          // padded members of the group
+    int w, slot, len;     // first word, first slot, words
+};
 // Items of one unit inside a CTA's share: plane words [i0, ip), fp16 octets [ip, i1).
 struct Seg {
     int u, i0, ip, i1;
@@ -254,13 +269,14 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t s_bar[kPhiBars + 2];  // Phi chunks, the two expert directories, the staged planes
     __shared__ Run s_run[kMaxItems];
+    __shared__ MetaRun s_mrun[kMaxItems];
     __shared__ UnitInfo s_unit[kMaxUnits];
     __shared__ Item s_item[kMaxItems];
     __shared__ MemberWord s_mw[kMaxItems];
     __shared__ Seg s_seg[kMaxItems];
     __shared__ uint2 s_desc[kMaxItems];  // plane word: (tables' shared address, 2^j bits)
     __shared__ float s_zpmw[kMaxItems];
-    __shared__ int s_ni, s_nmw, s_nseg, s_nrun, s_abort, s_bad;
+    __shared__ int s_ni, s_nmw, s_nseg, s_nrun, s_nmrun, s_abort, s_bad;
     __shared__ uint32_t s_stage_bytes;
     __shared__ unsigned long long s_bar_base;
 
@@ -275,7 +291,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     uint8_t* s_dir = smem + P.sm_dir;  // [projection][expert] directory entries
     uint8_t* s_phi = smem + P.sm_phi;
     uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);  // [item slot][d_pad]
-    uint8_t* s_mwd = smem + P.sm_mw;    // [member word]: idx u16[32] | scale u16[32] | amp f32[32]
+    // member-word metadata, one array each, 32 members per slot
+    uint16_t* s_midx = reinterpret_cast<uint16_t*>(smem + P.sm_mw);
+    uint16_t* s_mscl = s_midx + 32 * P.items_max;
+    float* s_mamp = reinterpret_cast<float*>(s_mscl + 32 * P.items_max);
     uint8_t* s_f16d = smem + P.sm_f16;  // [octet]: idx u16[8] | amp f32[8]
     float* s_c16 = reinterpret_cast<float*>(smem + P.sm_c16);  // [octet][8]
     // tables start on a 512-byte shared-memory boundary: one member word's 8
@@ -295,6 +314,11 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         s_bar_base = ld_relaxed_u64(P.barrier);
     }
     __syncthreads();  // the mbarriers are initialised
+    // Roles: warp 1 plans this CTA's share and hands it to the last kStageWarps
+    // warps, which issue the staging copies; the other warps compute z rows as
+    // the Phi chunks land.  The three run side by side.
+    const int nrw = nwarps - kStageWarps;  // warps before the staging warps
+    const bool row_warp = warp < nrw;
     if (tid == 0) {
         // both expert directories first: the routed units need them before anything else
         const uint32_t dir_bytes = (uint32_t)P.E * kDirEntryBytes;
@@ -409,6 +433,28 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             M.seg = (int16_t)seg;
             s_mw[slot_new] = M;
         }
+        {   // runs of member words in slot order: consecutive slots, same group, consecutive words
+            const unsigned below = bm & lt;
+            const int prev = below ? 31 - __clz(below) : 0;  // the previous slot's lane
+            const int pkey = __shfl_sync(0xffffffffu, key, prev);
+            const bool mcont = newmw && below != 0u && pkey == key - 1;
+            const unsigned bmc = __ballot_sync(0xffffffffu, mcont);
+            const unsigned bmr = bm & ~bmc;  // run starts
+            if ((bmr >> lane) & 1u) {
+                const unsigned after = lane == 31 ? 0u : ~((2u << lane) - 1u);
+                const unsigned nxt = bmr & after;
+                const unsigned span = nxt ? (after & ((1u << (__ffs(nxt) - 1)) - 1u)) : after;
+                const UnitInfo& U = s_unit[my_u];
+                MetaRun R;
+                R.meta = P.proj[U.p].blob + U.gbase[g];
+                R.np = U.np[g];
+                R.w = w;
+                R.slot = slot_new;
+                R.len = 1 + __popc(bm & span);
+                s_mrun[__popc(bmr & lt)] = R;
+            }
+            if (lane == 0) s_nmrun = __popc(bmr);
+        }
         if (newseg) {
             const unsigned above = bs & ~(lt | (1u << lane));
             const int i1 = above ? __ffs(above) - 1 : ni;
@@ -444,21 +490,17 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             s_stage_bytes = 4u * (uint32_t)P.d_pad * (uint32_t)__popc(bplane) + 256u * __popc(bm) + 48u * __popc(bf);
             s_bad = bad;
         }
+        named_barrier<2>(32 * (1 + kStageWarps));  // the plan is in shared memory: hand it to the staging warps
     }
-    __syncthreads();
-    const int ni = s_ni, nmw = s_nmw, nseg = s_nseg;
-    // The last kStageWarps warps issue the staging copies; their issue can stall
-    // behind the Phi traffic, so the z rows are left to the other warps.
-    const int nrw = nwarps - kStageWarps;  // row warps
-    const bool row_warp = warp < nrw;
 
     // ---- the outputs are sums of red.add contributions: each CTA zeroes a slice first ----
-    {
+    const int rw = warp == 0 ? 0 : warp - 1, nrw1 = nrw - 1;  // index and count of the z-row warps
+    if (row_warp && warp != 1) {
         const int nys = 2 * P.d_out;
         const int nye0 = P.proj[0].Ye ? P.K * P.d_out : 0, nye1 = P.proj[1].Ye ? P.K * P.d_out : 0;
         const int tot = nys + nye0 + nye1;
         const int a = share_begin(cta, tot, P.G), b = share_begin(cta + 1, tot, P.G);
-        for (int i = a + tid; row_warp && i < b; i += nrw * 32) {
+        for (int i = a + rw * 32 + lane; i < b; i += nrw1 * 32) {
             float* dst;
             if (i < P.d_out)
                 dst = P.proj[0].Ysum + i;
@@ -473,9 +515,11 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     }
 
     // ---- staging by the staging warp (bulk copies on one mbarrier): each run of plane
-    // words in one copy into [item slot][d_pad]; then each member word's idx, scale
-    // and amp, and each octet's idx and amp ----
+    // words in one copy into [item slot][d_pad]; each run of member words' idx, scale
+    // and amp in one copy per array; each octet's idx and amp ----
     if (!row_warp) {
+        named_barrier<2>(32 * (1 + kStageWarps));
+        const int ni = s_ni;
         const int st = threadIdx.x - nrw * 32, nst = kStageWarps * 32;
         const uint64_t stream = policy_evict_first();
         uint64_t* bar = &s_bar[kPhiBars + 1];
@@ -485,12 +529,12 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             const Run R = s_run[r];
             bulk_g2s(s_planes + (size_t)R.a * P.d_pad, R.ptr, 4u * (uint32_t)P.d_pad * (uint32_t)R.len, bar, stream);
         }
-        for (int m = st; m < nmw; m += nst) {
-            const MemberWord& M = s_mw[m];
-            uint8_t* dst = s_mwd + 256 * m;
-            bulk_g2s(dst, M.meta + 64ull * M.w, 64u, bar, stream);                              // idx
-            bulk_g2s(dst + 64, M.meta + 2ull * M.np + 64ull * M.w, 64u, bar, stream);            // scale
-            bulk_g2s(dst + 128, M.meta + 4ull * M.np + 128ull * M.w, 128u, bar, stream);         // amp
+        for (int r = st; r < s_nmrun; r += nst) {
+            const MetaRun R = s_mrun[r];
+            const uint32_t n = (uint32_t)R.len;
+            bulk_g2s(s_midx + 32 * R.slot, R.meta + 64ull * R.w, 64u * n, bar, stream);                // idx
+            bulk_g2s(s_mscl + 32 * R.slot, R.meta + 2ull * R.np + 64ull * R.w, 64u * n, bar, stream);  // scale
+            bulk_g2s(s_mamp + 32 * R.slot, R.meta + 4ull * R.np + 128ull * R.w, 128u * n, bar, stream);  // amp
         }
         for (int i = st; i < ni; i += nst) {
             const Item& it = s_item[i];
@@ -505,9 +549,9 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
 
     // ---- phase 1: z rows of this CTA (row warps), then the arrival at the grid barrier ----
     const unsigned long long G = (unsigned long long)P.G;
-    if (row_warp) {
+    if (row_warp && warp != 1) {
         bool ok = nrows == 0 || mbar_wait(&s_bar[0], 0);  // barrier 0 carries x
-        for (int rl = warp; ok && rl < nrows; rl += nrw) {
+        for (int rl = rw; ok && rl < nrows; rl += nrw1) {
             int bi = 0;
             while (bi + 1 < kPhiBars && rl >= (nrows * (bi + 1)) / kPhiBars) bi++;
             if (!mbar_wait(&s_bar[bi], 0)) {
@@ -538,7 +582,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         if (!ok) s_abort = 1;
         // The row warps' z rows and zeroed outputs are ordered before the arrival by
         // this CTA barrier and the cumulative release of the arrival itself.
-        asm volatile("bar.sync 1, %0;" ::"r"(nrw * 32) : "memory");
+        named_barrier<1>(nrw1 * 32);
         if (tid == 0) {
             for (int bi = 0; bi < kPhiBars; bi++)  // every bulk copy into this CTA's shared memory has landed
                 if (!mbar_wait(&s_bar[bi], 0)) s_abort = 1;
@@ -547,6 +591,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         }
     }
     __syncthreads();
+    const int ni = s_ni, nmw = s_nmw, nseg = s_nseg;
 
     // ---- grid barrier wait (bounded) ----
     // The counter is a multiple of G whenever no launch is in flight (it starts
@@ -576,12 +621,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     // ---- c_k = a_k s_k z_k, the tables and the zero-point share: a warp per member word ----
     for (int m = warp; m < nmw; m += nwarps) {
         const MemberWord M = s_mw[m];
-        const uint8_t* md = s_mwd + 256 * m;
-        const int k = reinterpret_cast<const uint16_t*>(md)[lane];
+        const int k = s_midx[32 * m + lane];
         float c = 0.0f;
         if (lane < M.nvalid && k < P.r)
-            c = reinterpret_cast<const float*>(md + 128)[lane] *
-                __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(md + 64)[lane])) *
+            c = s_mamp[32 * m + lane] * __half2float(__ushort_as_half(s_mscl[32 * m + lane])) *
                 __ldcg(P.zbuf + M.p * P.r + k);
         // entry e of table tb = the sum of c over the set bits of e (members 4 tb .. 4 tb + 3)
         const int e = lane & 15;

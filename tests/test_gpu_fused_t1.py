@@ -124,5 +124,5 @@ def test_chained_call_prefetch_changes_nothing(orc):
         x, ids, gw = case.x[:T].contiguous(), case.ids[:T].contiguous(), case.gate_w[:T].contiguous()
         a = lay.forward(x, ids, gw, want_experts=True)
         b = lay.forward(x, ids, gw, want_experts=True, next_layer=lay)
-        for k in a:
-            assert rel_err(a[k].cpu().numpy(), b[k].cpu().numpy()) <= 1e-6, (T, k)
+        for k in a:  # two runs of the atomic routed sum: the fp32 summation-order bound (~1e-5)
+            assert rel_err(a[k].cpu().numpy(), b[k].cpu().numpy()) <= 1e-5, (T, k)
