@@ -267,7 +267,7 @@ __host__ __device__ __forceinline__ int share_begin(int c, int Q, int G) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t s_bar[kPhiBars + 2];  // Phi chunks, the two expert directories, the staged planes
+    __shared__ uint64_t s_bar[kPhiBars + 3];  // Phi chunks, the two expert directories, the staged planes
     __shared__ Run s_run[kMaxItems];
     __shared__ MetaRun s_mrun[kMaxItems];
     __shared__ UnitInfo s_unit[kMaxUnits];
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     __shared__ uint2 s_desc[kMaxItems];  // plane word: (tables' shared address, 2^j bits)
     __shared__ float s_zpmw[kMaxItems];
     __shared__ int s_ni, s_nmw, s_nseg, s_nrun, s_nmrun, s_abort, s_bad;
-    __shared__ uint32_t s_stage_bytes;
+    __shared__ uint32_t s_stage_bytes, s_meta_bytes;
     __shared__ unsigned long long s_bar_base;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     // mbarriers and then issues the Phi rows and x (they need nothing) ----
     const int my_id = (warp == 1 && lane < P.U) ? P.ids[lane % P.K] : 0;
     if (tid == 0) {
-        for (int i = 0; i < kPhiBars + 2; i++) mbar_init(&s_bar[i], 1);
+        for (int i = 0; i < kPhiBars + 3; i++) mbar_init(&s_bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
         s_bar_base = ld_relaxed_u64(P.barrier);
@@ -393,6 +393,26 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             }
         }
         const bool plane = valid && it.nf == 0, oct = valid && it.nf > 0;
+        // runs of plane words: consecutive items whose words follow each other in the blob
+        const uint64_t my_ptr = (uint64_t)it.ptr;
+        const uint64_t prev_ptr = __shfl_up_sync(0xffffffffu, my_ptr, 1);
+        const int prev_plane = __shfl_up_sync(0xffffffffu, (int)plane, 1);
+        const bool cont = plane && lane > 0 && prev_plane && my_ptr == prev_ptr + 4ull * P.d_pad;
+        const unsigned bcont = __ballot_sync(0xffffffffu, cont), bplane = __ballot_sync(0xffffffffu, plane);
+        const unsigned brun = bplane & ~bcont;
+        if ((brun >> lane) & 1u) {
+            const unsigned stop = ~bcont & (lane == 31 ? 0u : ~((2u << lane) - 1u));  // first later item not continuing
+            Run R;
+            R.ptr = it.ptr;
+            R.a = lane;
+            R.len = (stop ? __ffs(stop) - 1 : 32) - lane;
+            s_run[__popc(brun & ((1u << lane) - 1u))] = R;
+        }
+        if (lane == 0) {
+            s_nrun = __popc(brun);
+            s_stage_bytes = 4u * (uint32_t)P.d_pad * (uint32_t)__popc(bplane);
+        }
+        named_barrier<2>(32 * (1 + kStageWarps));  // the plane runs are known: the staging warps copy them now
         // first item of the same member word, and whether any of them is plane 0
         int ref = lane, zp = 0;
         const int z0 = plane && jb == 0;
@@ -467,30 +487,14 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             S.ip = octs ? __ffs(octs) - 1 : i1;
             s_seg[seg] = S;
         }
-        // runs of plane words: consecutive items whose words follow each other in the blob
-        const uint64_t my_ptr = (uint64_t)it.ptr;
-        const uint64_t prev_ptr = __shfl_up_sync(0xffffffffu, my_ptr, 1);
-        const int prev_plane = __shfl_up_sync(0xffffffffu, (int)plane, 1);
-        const bool cont = plane && lane > 0 && prev_plane && my_ptr == prev_ptr + 4ull * P.d_pad;
-        const unsigned bcont = __ballot_sync(0xffffffffu, cont), bplane = __ballot_sync(0xffffffffu, plane);
-        const unsigned brun = bplane & ~bcont;
-        if ((brun >> lane) & 1u) {
-            const unsigned stop = ~bcont & (lane == 31 ? 0u : ~((2u << lane) - 1u));  // first later item not continuing
-            Run R;
-            R.ptr = it.ptr;
-            R.a = lane;
-            R.len = (stop ? __ffs(stop) - 1 : 32) - lane;
-            s_run[__popc(brun & lt)] = R;
-        }
         if (lane == 0) {
             s_ni = ni;
             s_nmw = __popc(bm);
             s_nseg = __popc(bs);
-            s_nrun = __popc(brun);
-            s_stage_bytes = 4u * (uint32_t)P.d_pad * (uint32_t)__popc(bplane) + 256u * __popc(bm) + 48u * __popc(bf);
+            s_meta_bytes = 256u * __popc(bm) + 48u * __popc(bf);
             s_bad = bad;
         }
-        named_barrier<2>(32 * (1 + kStageWarps));  // the plan is in shared memory: hand it to the staging warps
+        named_barrier<3>(32 * (1 + kStageWarps));  // the rest of the plan: member words and octets
     }
 
     // ---- the outputs are sums of red.add contributions: each CTA zeroes a slice first ----
@@ -519,7 +523,6 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     // and amp in one copy per array; each octet's idx and amp ----
     if (!row_warp) {
         named_barrier<2>(32 * (1 + kStageWarps));
-        const int ni = s_ni;
         const int st = threadIdx.x - nrw * 32, nst = kStageWarps * 32;
         const uint64_t stream = policy_evict_first();
         uint64_t* bar = &s_bar[kPhiBars + 1];
@@ -529,6 +532,11 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             const Run R = s_run[r];
             bulk_g2s(s_planes + (size_t)R.a * P.d_pad, R.ptr, 4u * (uint32_t)P.d_pad * (uint32_t)R.len, bar, stream);
         }
+        named_barrier<3>(32 * (1 + kStageWarps));
+        const int ni = s_ni;
+        bar = &s_bar[kPhiBars + 2];
+        if (st == 0) mbar_expect_tx(bar, s_meta_bytes);
+        __syncwarp();
         for (int r = st; r < s_nmrun; r += nst) {
             const MetaRun R = s_mrun[r];
             const uint32_t n = (uint32_t)R.len;
@@ -600,7 +608,8 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     const unsigned long long base = (s_bar_base / G) * G;
     if (tid == 0) {
         if (!grid_wait(P.barrier, base + G)) s_abort = 1;
-        if (!mbar_wait(&s_bar[kPhiBars + 1], 0)) s_abort = 1;  // the staged planes and metadata
+        if (!mbar_wait(&s_bar[kPhiBars + 1], 0)) s_abort = 1;  // the staged planes
+        if (!mbar_wait(&s_bar[kPhiBars + 2], 0)) s_abort = 1;  // and metadata
         if (s_bad && cta == 0 && P.status) atomicOr(P.status, BITSMOE_ST_BADEXPERT);
     }
     __syncthreads();
@@ -666,7 +675,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         for (int t = warp; t < P.n_rb; t += nwarps) {
             const uint32_t* pl = s_planes + t * kRB + lane;  // [item slot][d_pad]
             float acc = 0.0f;
-#pragma unroll 2
+#pragma unroll 4
             for (int i = S.i0; i < S.ip; i++) {
                 const uint2 d = s_desc[i];
                 const uint32_t word = pl[i * P.d_pad];
