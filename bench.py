@@ -468,27 +468,36 @@ def dominant_kernel(n_launches: int) -> str:
 
 
 def run_e2e(wl, cfg, T, n, dist):
+    """The public API as a decode loop calls it, one step after another: the step's
+    inputs (x, routing ids, gate weights) are packed in one pinned host buffer and
+    copied to the device in one transfer, the layer forward runs on views of that
+    buffer, and both routed sums (one [2][T][d_out] buffer) come back in one
+    transfer."""
     import torch
     m = wl.n_steps
-    xs = wl.x.cpu().pin_memory()
-    ids = wl.ids.cpu().pin_memory()
-    gws = wl.gw.cpu().pin_memory()
-    out_g = torch.empty((m, T, cfg.d_out), dtype=torch.float32).pin_memory()
-    out_u = torch.empty((m, T, cfg.d_out), dtype=torch.float32).pin_memory()
-    xd = torch.empty((T, cfg.d_in), dtype=torch.float16, device="cuda")
-    idd = torch.empty((T, cfg.top_k), dtype=torch.int32, device="cuda")
-    gwd = torch.empty((T, cfg.top_k), dtype=torch.float32, device="cuda")
+    xb, ib, gb = T * cfg.d_in * 2, T * cfg.top_k * 4, T * cfg.top_k * 4
+    o_i = (xb + 15) // 16 * 16
+    o_g = o_i + (ib + 15) // 16 * 16
+    nbytes = o_g + gb
+    host_in = torch.empty((m, nbytes), dtype=torch.uint8).pin_memory()
+    for s in range(m):
+        host_in[s, :xb] = wl.x[s].cpu().contiguous().view(torch.uint8).reshape(-1)
+        host_in[s, o_i:o_i + ib] = wl.ids[s].cpu().contiguous().view(torch.uint8).reshape(-1)
+        host_in[s, o_g:o_g + gb] = wl.gw[s].cpu().contiguous().view(torch.uint8).reshape(-1)
+    dev_in = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    xd = dev_in[:xb].view(torch.float16).view(T, cfg.d_in)
+    idd = dev_in[o_i:o_i + ib].view(torch.int32).view(T, cfg.top_k)
+    gwd = dev_in[o_g:o_g + gb].view(torch.float32).view(T, cfg.top_k)
+    dev_out = torch.empty((2, T, cfg.d_out), dtype=torch.float32, device="cuda")
+    out = {"Y_sum_gate": dev_out[0], "Y_sum_up": dev_out[1]}
+    host_out = torch.empty((m, 2, T, cfg.d_out), dtype=torch.float32).pin_memory()
     stream = torch.cuda.current_stream()
 
     def one(s):
         s = s % m
-        xd.copy_(xs[s], non_blocking=True)
-        idd.copy_(ids[s], non_blocking=True)
-        gwd.copy_(gws[s], non_blocking=True)
-        l = wl.layer_of(s)
-        o = wl.layers[l].forward(xd, idd, gwd, out=wl.out[l])
-        out_g[s].copy_(o["Y_sum_gate"], non_blocking=True)
-        out_u[s].copy_(o["Y_sum_up"], non_blocking=True)
+        dev_in.copy_(host_in[s], non_blocking=True)
+        wl.layers[wl.layer_of(s)].forward(xd, idd, gwd, out=out)
+        host_out[s].copy_(dev_out, non_blocking=True)
 
     for s in range(min(n, 50)):
         one(s)
@@ -503,11 +512,10 @@ def run_e2e(wl, cfg, T, n, dist):
     torch.cuda.synchronize()
     dist.barrier()
     sec = dist.max(ev0.elapsed_time(ev1)) / 1e3
-    h2d = T * cfg.d_in * 2 + T * cfg.top_k * 8
-    d2h = 2 * T * cfg.d_out * 4
-    return {"value": dist.world * n * T / sec, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": n, "how": "eager public-API loop: pinned H2D of x/ids/gate_w, SpectralMoELayer.forward, D2H of both "
-                               "Y_sum per step; CUDA events on the stream"}
+    return {"value": dist.world * n * T / sec, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": 2 * T * cfg.d_out * 4, "steps": n,
+            "how": "eager public-API loop, steps serialised: one pinned H2D of the step's packed x/ids/gate_w, "
+                   "SpectralMoELayer.forward on views of it, one D2H of both Y_sum; CUDA events on the stream"}
 
 
 def run_reference(args, dist):

@@ -178,4 +178,5 @@ struct bitsmoe_plan {
     uint32_t* counts;       // [E][8], groups in storage order, [7] = width 0
     uint32_t max_items;     // max over experts of (n16 + sum of words of bit-plane groups)
     uint32_t max_members_padded;  // max over experts of the padded member count (all groups)
+    uint32_t max_t1_items;  // max over experts of (words of bit-plane groups + fp16 octets)
 };

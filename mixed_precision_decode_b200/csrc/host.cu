@@ -40,11 +40,12 @@ static int finish_plan(bitsmoe_plan* p) {
     uint64_t base = p->header_bytes;
     p->max_items = 0;
     p->max_members_padded = 0;
+    p->max_t1_items = 0;
     for (int e = 0; e < E; e++) {
         const uint32_t* c = p->counts + 8 * (size_t)e;
         uint8_t* dir = p->header + kHeaderBytes + kDirEntryBytes * (uint64_t)e;
         uint64_t off = 0;
-        uint32_t items = 0, members = 0;
+        uint32_t items = 0, members = 0, t1_items = 0;
         for (int g = 0; g < kNumGroups; g++) {
             int b = group_width(g);
             put32(dir + 16 + 4 * g, (uint32_t)off);
@@ -53,6 +54,7 @@ static int finish_plan(bitsmoe_plan* p) {
             uint32_t np = (uint32_t)group_members_padded(b, c[g]);
             members += np;
             items += b == 16 ? c[g] : np / 32;
+            t1_items += b == 16 ? np / 8 : b * (np / 32);  // fp16 members padded to octets
         }
         put16(dir + 44 + 14, (uint16_t)c[7]);
         put64(dir, base);
@@ -60,6 +62,7 @@ static int finish_plan(bitsmoe_plan* p) {
         base += off;
         if (items > p->max_items) p->max_items = items;
         if (members > p->max_members_padded) p->max_members_padded = members;
+        if (t1_items > p->max_t1_items) p->max_t1_items = t1_items;
     }
     p->blob_bytes = base;
     uint8_t* h = p->header;

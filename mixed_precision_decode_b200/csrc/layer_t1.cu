@@ -27,6 +27,7 @@
 // has one grid barrier; the order of those additions, and so the last bits
 // of the outputs, can differ from run to run.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -727,6 +728,25 @@ static int g_num_sms = 0;
 static int g_max_smem = 0;
 static int g_static_smem = -1;
 
+// Largest dynamic shared memory size k_layer_t1 has been granted on each
+// device, so that a launch asks the runtime again only when it needs more.
+constexpr int kMaxDevices = 256;
+static std::atomic<int> g_smem_granted[kMaxDevices];
+
+static cudaError_t grant_smem(int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    if (cached && g_smem_granted[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(k_layer_t1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess || !cached) return e;
+    int prev = g_smem_granted[dev].load(std::memory_order_relaxed);
+    while (prev < bytes && !g_smem_granted[dev].compare_exchange_weak(prev, bytes)) {
+    }
+    return cudaSuccess;
+}
+
 static bool device_info() {
     if (g_num_sms > 0 && g_static_smem >= 0) return true;
     int dev;
@@ -739,20 +759,10 @@ static bool device_info() {
     return true;
 }
 
-// Work items (plane words + fp16 octets) of the largest expert of a plan.
-static int expert_items_max(const bitsmoe_plan* p) {
-    int best = 0;
-    for (int e = 0; e < p->dims.n_experts; e++) {
-        const uint32_t* c = p->counts + 8 * (size_t)e;
-        int pw = 0;
-        for (int g = 0; g < kNumGroups; g++) {
-            const int b = group_width(g);
-            if (b != 16) pw += b * (int)(group_members_padded(b, c[g]) / 32);
-        }
-        best = std::max(best, pw + (int)((c[0] + kF16Item - 1) / kF16Item));
-    }
-    return best;
-}
+// Work items (plane words + fp16 octets) of the largest expert of a plan,
+// counted once when the plan was built.
+static_assert(kF16Item == 8, "an fp16 item is one octet of the group's 8-member padding");
+static int expert_items_max(const bitsmoe_plan* p) { return (int)p->max_t1_items; }
 
 // Warps per CTA: every warp owns whole 32-row tiles, so take the count (8..24)
 // that leaves the fewest idle warp-tiles, the larger on a tie.
@@ -853,7 +863,7 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
     P.barrier = (unsigned long long*)ws;
     P.zbuf = (float*)(ws + L.ws_reserved);
 
-    cudaError_t e = cudaFuncSetAttribute(k_layer_t1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
+    cudaError_t e = grant_smem((int)L.smem);
     if (e != cudaSuccess) return set_cuda_error(e);
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)P.G);

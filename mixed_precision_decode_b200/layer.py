@@ -54,15 +54,34 @@ class SpectralMoELayer:
         assert gate.d_in == up.d_in and gate.top_k == up.top_k and gate.n_experts == up.n_experts
         self.gate, self.up = gate, up
         self._ws = {}
+        self._ios = {}
 
     def workspace(self, T: int) -> torch.Tensor:
-        n = B.layer_workspace_bytes(self.gate.plan, self.up.plan, T)
+        """The layer's workspace for T tokens, allocated on first use.  The plans
+        are immutable, so its size for a given T never changes."""
         ws = self._ws.get(T)
-        if ws is None or ws.numel() < n:
+        if ws is None:
+            n = B.layer_workspace_bytes(self.gate.plan, self.up.plan, T)
             # zero-filled once: its head keeps the fused path's counters between calls
             ws = torch.zeros(max(n, 256), dtype=torch.uint8, device=self.gate.blob.device)
             self._ws[T] = ws
         return ws
+
+    def _proj_ios(self, out: dict) -> tuple:
+        """The two projections' I/O descriptors for these output buffers, reused
+        while a caller keeps passing the same buffers (a decode loop)."""
+        key = tuple(None if t is None else t.data_ptr()
+                    for t in (out["Y_sum_gate"], out["Y_sum_up"], out.get("Z_gate"), out.get("Z_up"),
+                              out.get("Y_experts_gate"), out.get("Y_experts_up")))
+        ios = self._ios.get(key)
+        if ios is None:
+            ios = tuple(B.proj_io(p.plan, p.blob, p.phi_t, out[f"Y_sum_{name}"], out.get(f"Z_{name}"),
+                                  out.get(f"Y_experts_{name}"))
+                        for name, p in (("gate", self.gate), ("up", self.up)))
+            if len(self._ios) >= 64:
+                self._ios.clear()
+            self._ios[key] = ios
+        return ios
 
     def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, gate_w: torch.Tensor, out: dict | None = None,
                 want_experts: bool = False, want_z: bool = False, status: torch.Tensor | None = None,
@@ -81,10 +100,7 @@ class SpectralMoELayer:
                     out[f"Y_experts_{name}"] = torch.empty((T, p.top_k, p.d_out), dtype=torch.float32, device=dev)
                 if want_z:
                     out[f"Z_{name}"] = torch.empty((T, p.rank), dtype=torch.float32, device=dev)
-        ios = []
-        for name, p in (("gate", self.gate), ("up", self.up)):
-            ios.append(B.proj_io(p.plan, p.blob, p.phi_t, out[f"Y_sum_{name}"], out.get(f"Z_{name}"),
-                                 out.get(f"Y_experts_{name}")))
+        ios = self._proj_ios(out)
         ws = self.workspace(T)
         if next_layer is None:
             B.layer_forward(ios[0], ios[1], x, topk_ids, gate_w, T, ws, ws.numel(), status, stream)
