@@ -188,11 +188,16 @@ int bitsmoe_layer_launches(const bitsmoe_plan *gate, const bitsmoe_plan *up, int
  * sums.  X dev [T][d_in] fp16; topk_ids / gate_w as in bitsmoe_expert_forward
  * (shared by both projections).  The two plans must agree on d_in and top_k.
  * workspace dev (>= bitsmoe_layer_workspace_bytes, 256-byte aligned) must be
- * zero-filled once before its first use: its head holds counters of the fused
- * single-token path that every call leaves ready for the next one (after a
- * BITSMOE_ST_TIMEOUT status, zero it again).  Calls that share a workspace
- * must not overlap on the GPU.  With T = 1 the routed sum is formed in slot
- * order, so results do not depend on timing.  Errors: EINVAL, ESIZE, ECUDA. */
+ * zero-filled, all of it, once before its first use: its head holds the fused
+ * single-token path's state -- a launch counter and the z rows, each tagged
+ * with the launch that wrote it -- which every call (a timed-out one too)
+ * leaves ready for the next.  If it is ever cleared again, clear all of it:
+ * restarting the counter while z rows of earlier calls keep their tags could
+ * let a call take a stale row.  Calls that share a workspace must not overlap
+ * on the GPU.  With T = 1 the fused kernel adds the CTAs' partial rows with
+ * fp32 atomic additions, whose order, and so the last bits of Y_sum and
+ * Y_experts, can differ between runs; with T > 1 the routed sum is formed in
+ * slot order.  Errors: EINVAL, ESIZE, ECUDA. */
 int bitsmoe_layer_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,
                           const int32_t *topk_ids, const float *gate_w, int32_t T, void *workspace,
                           uint64_t workspace_bytes, int32_t *status, void *stream);
@@ -229,9 +234,9 @@ int bitsmoe_layer_forward_chained(const bitsmoe_proj_io *gate, const bitsmoe_pro
  *   gate, up, X, topk_ids, gate_w, status: as in bitsmoe_layer_forward with
  *   T = 1 (topk_ids / gate_w hold one row of top_k entries).
  * The first call on each device looks up the array's device address; make
- * that first call before any stream capture.  Every call clears the array's
- * counters and then uses it, so calls that overlap on the GPU (two streams,
- * two host threads) race and must be serialised by the caller.
+ * that first call before any stream capture.  The array starts zeroed and
+ * every call leaves it ready for the next, so calls that overlap on the GPU
+ * (two streams, two host threads) race and must be serialised by the caller.
  * Errors: EINVAL (dims, NULL or misaligned pointers), ESIZE (shapes the
  * single-launch kernel cannot hold, or scratch beyond 1 MiB), ECUDA. */
 int bitsmoe_layer_forward_t1_noalloc(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,

@@ -205,23 +205,20 @@ static uint64_t layer_ws(const bitsmoe_plan* g, const bitsmoe_plan* u, int T, co
 int layer_forward_fused_t1(const bitsmoe_proj_io* io[2], const uint16_t* X, const int32_t* ids, const float* gw,
                            void* workspace, uint64_t workspace_bytes, const uint16_t* const* next_phi, int32_t* status,
                            cudaStream_t s, bool* used);
-uint64_t layer_fused_t1_workspace(const bitsmoe_plan* g, const bitsmoe_plan* u);
 uint64_t layer_fused_t1_reserved(const bitsmoe_plan* g, const bitsmoe_plan* u);
 }  // namespace bitsmoe
 
-// Layer workspace = [fused-path counters (persistent) | per-call region].
+// Layer workspace = [fused single-token path's state (persistent) | per-call region of the other paths].
 BITSMOE_API uint64_t bitsmoe_layer_workspace_bytes(const bitsmoe_plan* gate, const bitsmoe_plan* up, int32_t T) {
     if (!gate || !up || T < 0) return 0;
     const uint64_t head = layer_fused_t1_reserved(gate, up);
-    uint64_t a = layer_ws(gate, up, T, nullptr, nullptr, nullptr);
-    uint64_t b = T == 1 ? layer_fused_t1_workspace(gate, up) : 0;
-    return head + (a > b ? a : b);
+    return head + layer_ws(gate, up, T, nullptr, nullptr, nullptr);
 }
 
 BITSMOE_API int bitsmoe_layer_launches(const bitsmoe_plan* gate, const bitsmoe_plan* up, int32_t T) {
     if (!gate || !up || T < 0) return BITSMOE_EINVAL;
     if (T == 0) return 0;
-    if (T == 1 && layer_fused_t1_workspace(gate, up) > 0) return 1;
+    if (T == 1 && layer_fused_t1_reserved(gate, up) > 0) return 1;
     return 7;  // route, then per projection: shared projection, experts, combine
 }
 

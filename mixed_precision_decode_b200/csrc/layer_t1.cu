@@ -8,11 +8,13 @@
 //                      - sum_b (2^b - 1)/2 sum_{k in G_b} c_k,  c_k = a_k s_k z_k.
 //
 // Design for B200 at one token.  The step moves ~24 MB (Phi of both
-// projections dominates) and has one grid-wide dependency (every expert row
-// needs all of z).  Every CTA issues its HBM reads at launch -- its slice of
-// Phi rows by TMA bulk copies, its share of the routed bit planes and their
-// metadata by cp.async -- computes its z rows and meets the other CTAs at a
-// bounded grid barrier.
+// projections dominates) and one grid-wide dependency (expert rows need z
+// rows that other CTAs compute).  Every CTA issues its HBM reads at launch --
+// its slice of Phi rows, its share of the routed bit planes and their
+// metadata, all by bulk copies -- and computes its z rows.  There is no grid
+// barrier: each z row is published as one 64-bit word carrying the launch's
+// tag next to the value, and a CTA polls exactly the z words its members need,
+// so the wait and the gather are one L2 round trip.
 //
 // The expert work is cut by COLUMNS: the routed units' plane words (one word
 // = one bit plane of 32 members, over all rows) and octets of fp16 members
@@ -23,9 +25,9 @@
 // over 32 members of one plane word uses eight 16-entry tables (one per
 // nibble), one shared-memory lookup per 4 bits.  Each CTA adds its rows of
 // every unit it touched (with its share of the zero-point term subtracted) to
-// Y_e and, times the gate weight, to Y_sum with fp32 red.add, so the kernel
-// has one grid barrier; the order of those additions, and so the last bits
-// of the outputs, can differ from run to run.
+// Y_e and, times the gate weight, to Y_sum with fp32 red.add, after acquiring
+// the tags the CTAs that zeroed the outputs published; the order of those
+// additions, and so the last bits of the outputs, can differ from run to run.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -43,6 +45,11 @@ constexpr int kF16Item = 8;       // fp16 members per item
 constexpr int kStageWarps = 1;    // warps that issue the plane and metadata copies
 constexpr int kPhiBars = 4;       // mbarriers over the Phi slice
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded waits: 2 s, then BITSMOE_ST_TIMEOUT
+constexpr int kTagBar = kPhiBars + 3;  // mbarrier that hands this launch's tag to the row warps
+constexpr int kMaxZeroCtas = 16;       // CTAs that zero the outputs (each publishes a tag)
+constexpr int kZeroSliceFloats = 16384;  // outputs zeroed per zeroing CTA, at least
+// workspace head: [0] launch counter, [1 .. kMaxZeroCtas] the zeroing CTAs' tags
+static_assert(8 * (1 + kMaxZeroCtas) <= 256, "the workspace head is 256 bytes");
 
 struct T1Proj {
     const uint8_t* blob;
@@ -59,10 +66,12 @@ struct T1Params {
     const int32_t* ids;
     const float* gw;
     int32_t* status;
-    unsigned long long* barrier;  // persistent, zero-initialised once; G arrivals per launch
-    float* zbuf;                  // [2][r]
+    unsigned long long* launches;   // persistent, zero-initialised once; every CTA adds 1 per launch
+    unsigned long long* zero_tags;  // [n_zero]: tag of the last launch whose outputs each zeroing CTA cleared
+    unsigned long long* zbuf;       // [2][r] z rows, each (launch tag << 32) | fp32 bits
     int d_in, d_out, d_pad, r, K, E, U;
     int n_rb, G;
+    int n_zero;     // CTAs that zero the outputs (1 .. kMaxZeroCtas)
     int items_max;  // work items per CTA (upper bound over every routing)
     // dynamic shared-memory layout (byte offsets)
     uint32_t sm_x, sm_dir, sm_phi, sm_planes, sm_mw, sm_f16, sm_c16, sm_tab, sm_end;
@@ -81,6 +90,9 @@ __device__ __forceinline__ long long globaltimer() {
 }
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -156,16 +168,36 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void red_add_release_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-// Bounded spin until the grid-barrier counter reaches target; false on timeout.
-__device__ __forceinline__ bool grid_wait(const unsigned long long* ctr, unsigned long long target) {
-    if (ld_acquire_u64(ctr) >= target) return true;
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Bounded spin until *p holds tag (acquire); false on timeout.
+__device__ __forceinline__ bool tag_wait(const unsigned long long* p, unsigned long long tag) {
+    if (ld_acquire_u64(p) == tag) return true;
     const long long t0 = globaltimer();
-    while (ld_acquire_u64(ctr) < target)
+    while (ld_acquire_u64(p) != tag)
         if (globaltimer() - t0 > kWaitLimitNs) return false;
     return true;
+}
+// z row k of this launch: a z word is one 64-bit store of (tag << 32) | value,
+// so the load that sees this launch's tag also sees its value.  Polls (bounded;
+// on timeout, or once another thread of the CTA timed out, sets *timed_out and
+// returns 0).
+__device__ __forceinline__ float z_poll(const unsigned long long* w, uint32_t tag, volatile int* timed_out) {
+    unsigned long long v = ld_relaxed_u64(w);
+    if ((uint32_t)(v >> 32) != tag) {
+        const long long t0 = globaltimer();
+        while ((uint32_t)((v = ld_relaxed_u64(w)) >> 32) != tag) {
+            if (*timed_out || globaltimer() - t0 > kWaitLimitNs) {
+                *timed_out = 1;
+                return 0.0f;
+            }
+        }
+    }
+    return __uint_as_float((uint32_t)v);
 }
 
 // ---------------------------------------------------------------------------
@@ -268,7 +300,7 @@ __host__ __device__ __forceinline__ int share_begin(int c, int Q, int G) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t s_bar[kPhiBars + 3];  // Phi chunks, the two expert directories, the staged planes
+    __shared__ uint64_t s_bar[kPhiBars + 4];  // Phi chunks, the expert directories, planes, metadata, tag
     __shared__ Run s_run[kMaxItems];
     __shared__ MetaRun s_mrun[kMaxItems];
     __shared__ UnitInfo s_unit[kMaxUnits];
@@ -278,8 +310,9 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     __shared__ uint2 s_desc[kMaxItems];  // plane word: (tables' shared address, 2^j bits)
     __shared__ float s_zpmw[kMaxItems];
     __shared__ int s_ni, s_nmw, s_nseg, s_nrun, s_nmrun, s_abort, s_bad;
+    __shared__ volatile int s_zto;  // a z poll timed out
     __shared__ uint32_t s_stage_bytes, s_meta_bytes;
-    __shared__ unsigned long long s_bar_base;
+    __shared__ uint32_t s_tag;      // this launch's tag (1 .. 2^32 - 1)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nthreads = blockDim.x, nwarps = nthreads >> 5;
@@ -309,10 +342,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     // mbarriers and then issues the Phi rows and x (they need nothing) ----
     const int my_id = (warp == 1 && lane < P.U) ? P.ids[lane % P.K] : 0;
     if (tid == 0) {
-        for (int i = 0; i < kPhiBars + 3; i++) mbar_init(&s_bar[i], 1);
+        for (int i = 0; i < kPhiBars + 4; i++) mbar_init(&s_bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
-        s_bar_base = ld_relaxed_u64(P.barrier);
+        s_zto = 0;
     }
     __syncthreads();  // the mbarriers are initialised
     // Roles: warp 1 plans this CTA's share and hands it to the last kStageWarps
@@ -340,6 +373,14 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                 rr += n;
             }
         }
+        // This launch's tag.  Every launch adds exactly G to the counter (one per
+        // CTA, whatever happens later), so before this CTA's addition it holds G
+        // times the number of earlier launches n plus fewer than G of this one's.
+        // The tag, n mod (2^32 - 1) plus 1, is never 0 (a zero-filled z word) and
+        // never that of the launch before.
+        const unsigned long long before = atomicAdd(P.launches, 1ull);
+        s_tag = (uint32_t)((before / (unsigned long long)P.G) % 0xFFFFFFFFull) + 1u;
+        mbar_arrive(&s_bar[kTagBar]);  // publishes s_tag to the row warps
     }
 
     // ---- routed units and this CTA's share (warp 1; one lane per unit, then per item).
@@ -498,13 +539,15 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         named_barrier<3>(32 * (1 + kStageWarps));  // the rest of the plan: member words and octets
     }
 
-    // ---- the outputs are sums of red.add contributions: each CTA zeroes a slice first ----
+    // ---- the outputs are sums of red.add contributions: the first n_zero CTAs zero
+    // them and then publish this launch's tag; every CTA acquires those tags before
+    // its first addition ----
     const int rw = warp == 0 ? 0 : warp - 1, nrw1 = nrw - 1;  // index and count of the z-row warps
-    if (row_warp && warp != 1) {
+    if (cta < P.n_zero && row_warp && warp != 1) {
         const int nys = 2 * P.d_out;
         const int nye0 = P.proj[0].Ye ? P.K * P.d_out : 0, nye1 = P.proj[1].Ye ? P.K * P.d_out : 0;
         const int tot = nys + nye0 + nye1;
-        const int a = share_begin(cta, tot, P.G), b = share_begin(cta + 1, tot, P.G);
+        const int a = share_begin(cta, tot, P.n_zero), b = share_begin(cta + 1, tot, P.n_zero);
         for (int i = a + rw * 32 + lane; i < b; i += nrw1 * 32) {
             float* dst;
             if (i < P.d_out)
@@ -517,6 +560,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                 dst = P.proj[1].Ye + (i - nys - nye0);
             *dst = 0.0f;
         }
+        // the row warps' zeros are ordered before the tag by this CTA barrier and
+        // the cumulative release of the store (thread 0 wrote s_tag itself)
+        named_barrier<4>(nrw1 * 32);
+        if (tid == 0) st_release_u64(P.zero_tags + cta, (unsigned long long)s_tag);
     }
 
     // ---- staging by the staging warp (bulk copies on one mbarrier): each run of plane
@@ -556,10 +603,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         }
     }
 
-    // ---- phase 1: z rows of this CTA (row warps), then the arrival at the grid barrier ----
-    const unsigned long long G = (unsigned long long)P.G;
+    // ---- phase 1: z rows of this CTA (row warps), each published with this launch's tag ----
     if (row_warp && warp != 1) {
-        bool ok = nrows == 0 || mbar_wait(&s_bar[0], 0);  // barrier 0 carries x
+        bool ok = nrows == 0 || (mbar_wait(&s_bar[kTagBar], 0) && mbar_wait(&s_bar[0], 0));  // 0 carries x
+        const unsigned long long tag_hi = (unsigned long long)s_tag << 32;
         for (int rl = rw; ok && rl < nrows; rl += nrw1) {
             int bi = 0;
             while (bi + 1 < kPhiBars && rl >= (nrows * (bi + 1)) / kPhiBars) bi++;
@@ -584,31 +631,24 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             acc = warp_sum(acc);
             if (lane == 0) {
                 const int rr = row0 + rl, p = rr / P.r, k = rr - p * P.r;
-                P.zbuf[rr] = acc;
+                st_relaxed_u64(P.zbuf + rr, tag_hi | __float_as_uint(acc));
                 if (P.proj[p].Z) P.proj[p].Z[k] = acc;
             }
         }
         if (!ok) s_abort = 1;
-        // The row warps' z rows and zeroed outputs are ordered before the arrival by
-        // this CTA barrier and the cumulative release of the arrival itself.
         named_barrier<1>(nrw1 * 32);
-        if (tid == 0) {
+        if (tid == 0)
             for (int bi = 0; bi < kPhiBars; bi++)  // every bulk copy into this CTA's shared memory has landed
                 if (!mbar_wait(&s_bar[bi], 0)) s_abort = 1;
-            __threadfence();
-            red_add_release_u64(P.barrier, 1ull);  // arrive
-        }
     }
     __syncthreads();
     const int ni = s_ni, nmw = s_nmw, nseg = s_nseg;
+    const uint32_t tag = s_tag;
 
-    // ---- grid barrier wait (bounded) ----
-    // The counter is a multiple of G whenever no launch is in flight (it starts
-    // at zero and every launch adds exactly G), so the value read at start
-    // rounded down to a multiple of G is this launch's base.
-    const unsigned long long base = (s_bar_base / G) * G;
+    // ---- the outputs are zeroed, the planes and metadata have landed (bounded waits) ----
     if (tid == 0) {
-        if (!grid_wait(P.barrier, base + G)) s_abort = 1;
+        for (int z = 0; z < P.n_zero; z++)
+            if (!tag_wait(P.zero_tags + z, (unsigned long long)tag)) s_abort = 1;
         if (!mbar_wait(&s_bar[kPhiBars + 1], 0)) s_abort = 1;  // the staged planes
         if (!mbar_wait(&s_bar[kPhiBars + 2], 0)) s_abort = 1;  // and metadata
         if (s_bad && cta == 0 && P.status) atomicOr(P.status, BITSMOE_ST_BADEXPERT);
@@ -618,15 +658,6 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
         return;
     }
-    // Every CTA has read its Phi: HBM is free while the experts are evaluated, so
-    // pull this CTA's rows of the next layer's Phi into L2 for the next call.
-    if (tid == 0 && P.next_phi[0] && P.next_phi[1])
-        for (int rr = row0; rr < row1;) {
-            const int p = rr / P.r, k = rr - p * P.r;
-            const int n = min(row1 - rr, P.r - k);
-            bulk_prefetch_l2(P.next_phi[p] + (size_t)k * P.d_in, (uint32_t)n * row_bytes);
-            rr += n;
-        }
 
     // ---- c_k = a_k s_k z_k, the tables and the zero-point share: a warp per member word ----
     for (int m = warp; m < nmw; m += nwarps) {
@@ -635,7 +666,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         float c = 0.0f;
         if (lane < M.nvalid && k < P.r)
             c = s_mamp[32 * m + lane] * __half2float(__ushort_as_half(s_mscl[32 * m + lane])) *
-                __ldcg(P.zbuf + M.p * P.r + k);
+                z_poll(P.zbuf + M.p * P.r + k, tag, &s_zto);
         // entry e of table tb = the sum of c over the set bits of e (members 4 tb .. 4 tb + 3)
         const int e = lane & 15;
 #pragma unroll
@@ -658,10 +689,24 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         const int k = reinterpret_cast<const uint16_t*>(fd)[m];
         float c = 0.0f;
         if (m < it.nf && k < P.r)
-            c = reinterpret_cast<const float*>(fd + 16)[m] * __ldcg(P.zbuf + s_unit[it.u].p * P.r + k);
+            c = reinterpret_cast<const float*>(fd + 16)[m] * z_poll(P.zbuf + s_unit[it.u].p * P.r + k, tag, &s_zto);
         s_c16[kF16Item * it.slot + m] = c;
     }
     __syncthreads();
+    if (s_zto) {
+        if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
+        return;
+    }
+    // This CTA has every z row it needs, so the Phi reads of this launch are all
+    // but done: HBM is free while the experts are evaluated, so pull this CTA's
+    // rows of the next layer's Phi into L2 for the next call.
+    if (tid == 0 && P.next_phi[0] && P.next_phi[1])
+        for (int rr = row0; rr < row1;) {
+            const int p = rr / P.r, k = rr - p * P.r;
+            const int n = min(row1 - rr, P.r - k);
+            bulk_prefetch_l2(P.next_phi[p] + (size_t)k * P.d_in, (uint32_t)n * row_bytes);
+            rr += n;
+        }
 
     // ---- lookups: warps own 32-row tiles; a segment's rows go to Y_e and, times g, to Y_sum ----
     for (int s = 0; s < nseg; s++) {
@@ -719,7 +764,6 @@ struct T1Layout {
     bool ok;
     T1Params P;
     uint64_t ws_reserved;  // persistent counter at the start of the workspace
-    uint64_t ws_bytes;
     size_t smem;
     int threads;
 };
@@ -819,21 +863,16 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     L.smem = P.sm_end;
     if (L.smem + (size_t)g_static_smem > (size_t)g_max_smem) return L;
     L.threads = 32 * choose_warps(P.n_rb);
-    // workspace: [barrier counter] persistent at the head, then z
-    L.ws_reserved = 256;
-    L.ws_bytes = roundup(4ull * 2 * P.r, 256);  // bytes after the reserved head
+    // workspace: the launch counter and the zeroing CTAs' tags (a 256-byte head),
+    // then the tagged z rows.  All of it persists between calls (a stale z word
+    // must never carry a live tag), so other paths work after it.
+    L.ws_reserved = 256 + roundup(8ull * 2 * P.r, 256);
     L.ok = true;
     return L;
 }
 
-// Bytes the fused path uses after the reserved head (0 when it does not apply).
-uint64_t layer_fused_t1_workspace(const bitsmoe_plan* g, const bitsmoe_plan* u) {
-    T1Layout L = t1_layout(g, u);
-    return L.ok ? L.ws_bytes : 0;
-}
-
 // Bytes at the head of a layer workspace that hold the fused path's
-// persistent counter (0 when it does not apply).
+// persistent state: its counters and tagged z rows (0 when it does not apply).
 uint64_t layer_fused_t1_reserved(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     T1Layout L = t1_layout(g, u);
     return L.ok ? L.ws_reserved : 0;
@@ -844,7 +883,7 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
                            cudaStream_t s, bool* used) {
     *used = false;
     T1Layout L = t1_layout(io[0]->plan, io[1]->plan);
-    if (!L.ok || workspace_bytes < L.ws_reserved + L.ws_bytes) return BITSMOE_OK;
+    if (!L.ok || workspace_bytes < L.ws_reserved) return BITSMOE_OK;
     T1Params P = L.P;
     for (int j = 0; j < 2; j++) {
         P.proj[j].blob = (const uint8_t*)io[j]->blob;
@@ -860,8 +899,13 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
     P.gw = gw;
     P.status = status;
     uint8_t* ws = (uint8_t*)workspace;
-    P.barrier = (unsigned long long*)ws;
-    P.zbuf = (float*)(ws + L.ws_reserved);
+    P.launches = (unsigned long long*)ws;
+    P.zero_tags = P.launches + 1;
+    P.zbuf = (unsigned long long*)(ws + 256);
+    // enough zeroing CTAs that each clears at least kZeroSliceFloats outputs
+    const long long n_out = (long long)P.d_out * (2 + (io[0]->Y_experts ? P.K : 0) + (io[1]->Y_experts ? P.K : 0));
+    P.n_zero = (int)std::min<long long>({(n_out + kZeroSliceFloats - 1) / kZeroSliceFloats, kMaxZeroCtas, P.G});
+    P.n_zero = std::max(P.n_zero, 1);
 
     cudaError_t e = grant_smem((int)L.smem);
     if (e != cudaSuccess) return set_cuda_error(e);
@@ -885,10 +929,9 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
 
 // ---------------------------------------------------------------------------
 // Single-token layer forward with library-owned scratch, for callers that
-// cannot allocate device memory.  The scratch (the fused kernel's grid-barrier
-// counter, z of both projections and the partial rows of the routed sum)
-// lives in one fixed static device array instead of a
-// caller-provided workspace.
+// cannot allocate device memory.  The scratch (the fused kernel's launch
+// counter, its zeroing tags and the tagged z rows of both projections) lives
+// in one fixed static device array instead of a caller-provided workspace.
 // ---------------------------------------------------------------------------
 namespace bitsmoe {
 
@@ -936,17 +979,17 @@ BITSMOE_API int bitsmoe_layer_forward_t1_noalloc(const bitsmoe_proj_io* gate, co
     if ((uintptr_t)X % 16) return BITSMOE_EINVAL;
     // shapes the single-launch kernel cannot hold, or whose scratch exceeds the array
     const uint64_t head = layer_fused_t1_reserved(pg, pu);
-    const uint64_t rest = layer_fused_t1_workspace(pg, pu);
-    if (head == 0 || rest == 0 || head + rest > kNoAllocScratchBytes) return BITSMOE_ESIZE;
+    if (head == 0 || head > kNoAllocScratchBytes) return BITSMOE_ESIZE;
     void* scratch = nullptr;
     int rc = noalloc_scratch(&scratch);
     if (rc) return rc;
     cudaStream_t s = (cudaStream_t)stream;
-    // the counters must start at zero; the array keeps whatever the last call left
-    cudaError_t e = cudaMemsetAsync(scratch, 0, head, s);
-    if (e != cudaSuccess) return set_cuda_error(e);
+    // The array starts zeroed and every call leaves it ready for the next one
+    // (the counter a multiple of the grid, each z word tagged with the launch
+    // that wrote it), so it is never cleared: clearing it would restart the
+    // tags while z words of earlier calls still carry them.
     bool used = false;
-    rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, scratch, head + rest, nullptr, status, s, &used);
+    rc = layer_forward_fused_t1(io, X, topk_ids, gate_w, scratch, head, nullptr, status, s, &used);
     if (rc) return rc;
     return used ? BITSMOE_OK : BITSMOE_ESIZE;
 }

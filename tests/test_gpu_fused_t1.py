@@ -52,9 +52,9 @@ def test_fused_t1_against_oracle(name, orc):
 
 
 def test_fused_t1_repeated_calls_interleaved_with_batches():
-    """Many single-token calls on one workspace (its counters carry over from
-    call to call), interleaved with batched calls that use the same workspace,
-    all agree with the general kernels to fp32 rounding."""
+    """Many single-token calls on one workspace (its counter and tagged z rows
+    carry over from call to call), interleaved with batched calls, all agree
+    with the general kernels to fp32 rounding."""
     case = get_case("qwen_t64")
     lay = case.layer
     gen = torch.Generator(device="cuda").manual_seed(5)
@@ -76,6 +76,43 @@ def test_fused_t1_repeated_calls_interleaved_with_batches():
     b = _one(case, 3)
     for proj in ("gate", "up"):
         assert rel_err(a[f"Y_sum_{proj}"].cpu().numpy(), b[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-5
+
+
+def test_fused_t1_workspace_shared_with_batches_across_tag_wrap():
+    """One workspace shared by single-token and 5-token calls (the batched path
+    writes its scratch after the fused path's persistent state), with the launch
+    counter started just below the point where the 32-bit launch tag wraps: every
+    single-token result matches the general kernels, and the counter advances by
+    exactly one grid per single-token launch."""
+    case = get_case("qwen_t64")
+    pg, pu = case.proj["gate"], case.proj["up"]
+    G = torch.cuda.get_device_properties(0).multi_processor_count
+    n = max(B.layer_workspace_bytes(pg.plan, pu.plan, T) for T in (1, 5))
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    start = G * (2 ** 32 - 3)  # tags of the next launches: 2^32 - 2, 2^32 - 1, 1, 2, ...
+    ws[:8].view(torch.int64)[0] = start
+    d_out = case.cfg.d_out
+    n_t1 = 0
+    for it in range(8):
+        t = it % case.cfg.tokens
+        out = {k: torch.full((1, d_out), float("nan"), device="cuda") for k in ("Y_sum_gate", "Y_sum_up")}
+        ios = [B.proj_io(p.plan, p.blob, p.phi_t, out[f"Y_sum_{name}"]) for name, p in (("gate", pg), ("up", pu))]
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        B.layer_forward(ios[0], ios[1], case.x[t:t + 1].contiguous(), case.ids[t:t + 1].contiguous(),
+                        case.gate_w[t:t + 1].contiguous(), 1, ws, n, st)
+        assert B.read_status(st) == 0
+        n_t1 += 1
+        ref = _general(case, t)
+        for proj in ("gate", "up"):
+            assert rel_err(out[f"Y_sum_{proj}"].cpu().numpy(), ref[f"Y_sum_{proj}"].cpu().numpy()) <= 1e-5, (it, proj)
+        if it % 2 == 1:  # a batched call over the same workspace
+            outb = {k: torch.empty((5, d_out), device="cuda") for k in ("Y_sum_gate", "Y_sum_up")}
+            iob = [B.proj_io(p.plan, p.blob, p.phi_t, outb[f"Y_sum_{name}"]) for name, p in (("gate", pg), ("up", pu))]
+            B.layer_forward(iob[0], iob[1], case.x[:5].contiguous(), case.ids[:5].contiguous(),
+                            case.gate_w[:5].contiguous(), 5, ws, n, st)
+            assert B.read_status(st) == 0
+    torch.cuda.synchronize()
+    assert int(ws[:8].view(torch.int64)[0]) == start + n_t1 * G
 
 
 def test_fused_t1_bad_expert_id():
