@@ -571,6 +571,12 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     // and amp in one copy per array; each octet's idx and amp ----
     if (!row_warp) {
         named_barrier<2>(32 * (1 + kStageWarps));
+        // A CTA's bulk copies land in about the order they are issued, so copies
+        // issued now would land after this CTA's Phi rows anyway; issued now they
+        // would also take HBM time from other CTAs' Phi rows, which every CTA
+        // waits for.  So they are issued once this CTA's last Phi chunk has landed.
+        const bool phi_ok = mbar_wait(&s_bar[kPhiBars - 1], 0);
+        if (!phi_ok) s_abort = 1;
         const int st = threadIdx.x - nrw * 32, nst = kStageWarps * 32;
         const uint64_t stream = policy_evict_first();
         uint64_t* bar = &s_bar[kPhiBars + 1];
