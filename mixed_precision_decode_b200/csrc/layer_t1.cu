@@ -289,6 +289,23 @@ struct Seg {
     int u, i0, ip, i1;
 };
 
+// acc0 += the products of the low halves of the four fp16 pairs of a and b,
+// acc1 += those of the high halves: mixed-precision FMAs (fp16 operands, exact
+// in fp32; fp32 addend), so no fp16 value is converted on its own.
+__device__ __forceinline__ void dot8_f16(const uint4 a, const uint4 b, float& acc0, float& acc1) {
+    asm("{\n"
+        " .reg .f16 a0, a1, a2, a3, a4, a5, a6, a7, b0, b1, b2, b3, b4, b5, b6, b7;\n"
+        " mov.b32 {a0, a1}, %2;\n mov.b32 {a2, a3}, %3;\n mov.b32 {a4, a5}, %4;\n mov.b32 {a6, a7}, %5;\n"
+        " mov.b32 {b0, b1}, %6;\n mov.b32 {b2, b3}, %7;\n mov.b32 {b4, b5}, %8;\n mov.b32 {b6, b7}, %9;\n"
+        " fma.rn.f32.f16 %0, a0, b0, %0;\n fma.rn.f32.f16 %1, a1, b1, %1;\n"
+        " fma.rn.f32.f16 %0, a2, b2, %0;\n fma.rn.f32.f16 %1, a3, b3, %1;\n"
+        " fma.rn.f32.f16 %0, a4, b4, %0;\n fma.rn.f32.f16 %1, a5, b5, %1;\n"
+        " fma.rn.f32.f16 %0, a6, b6, %0;\n fma.rn.f32.f16 %1, a7, b7, %1;\n"
+        "}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
+}
+
 // Items [q0, q1) of CTA c out of Q: an equal contiguous share.  c * Q stays
 // below 2^32 for every shape the fused path takes (the host checks it).
 __host__ __device__ __forceinline__ int share_begin(int c, int Q, int G) {
@@ -622,19 +639,9 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             }
             const uint4* rowv = reinterpret_cast<const uint4*>(s_phi + (size_t)rl * row_bytes);
             const uint4* xv = reinterpret_cast<const uint4*>(s_x);
-            float acc = 0.0f;
-            for (int i8 = lane; i8 < P.d_in / 8; i8 += 32) {
-                const uint4 a = rowv[i8], b = xv[i8];
-                const __half2* ha = reinterpret_cast<const __half2*>(&a);
-                const __half2* hb = reinterpret_cast<const __half2*>(&b);
-#pragma unroll
-                for (int h = 0; h < 4; h++) {
-                    const float2 fa = __half22float2(ha[h]), fb = __half22float2(hb[h]);
-                    acc = fmaf(fa.x, fb.x, acc);
-                    acc = fmaf(fa.y, fb.y, acc);
-                }
-            }
-            acc = warp_sum(acc);
+            float acc = 0.0f, acc1 = 0.0f;
+            for (int i8 = lane; i8 < P.d_in / 8; i8 += 32) dot8_f16(rowv[i8], xv[i8], acc, acc1);
+            acc = warp_sum(acc + acc1);
             if (lane == 0) {
                 const int rr = row0 + rl, p = rr / P.r, k = rr - p * P.r;
                 st_relaxed_u64(P.zbuf + rr, tag_hi | __float_as_uint(acc));
