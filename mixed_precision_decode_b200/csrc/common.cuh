@@ -165,6 +165,9 @@ struct RouteWS {
     int32_t* active;   // [E]   experts with at least one pair, ascending
     int32_t* nactive;  // [1]
     int32_t* pairs;    // [T*K] pair index t*K + j, grouped by expert
+    float* cvals;      // [T*K][ldc] c of every member of each pair's expert (multi-token path)
+    float* zp;         // [T*K] each pair's zero-point total
+    uint32_t ldc;      // floats per c row
 };
 }  // namespace bitsmoe
 

@@ -31,13 +31,18 @@ struct WsCursor {
     }
 };
 
-static RouteWS take_route(WsCursor& c, int E, int T, int K) {
+uint32_t cvals_ldc(const bitsmoe_plan* p);
+
+static RouteWS take_route(WsCursor& c, int E, int T, int K, uint32_t ldc) {
     RouteWS r;
     r.count = (int32_t*)c.take(4ull * E);
     r.start = (int32_t*)c.take(4ull * (E + 1));
     r.active = (int32_t*)c.take(4ull * E);
     r.nactive = (int32_t*)c.take(4);
     r.pairs = (int32_t*)c.take(4ull * (uint64_t)T * K + 4);
+    r.ldc = ldc;
+    r.cvals = (float*)c.take(4ull * (uint64_t)T * K * ldc);
+    r.zp = (float*)c.take(4ull * (uint64_t)T * K + 4);
     return r;
 }
 
@@ -121,14 +126,14 @@ __global__ void k_combine(const int32_t* __restrict__ ids, const float* __restri
     }
 }
 
-int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, int T, const RouteWS& rw, float* Ye,
-                     int32_t* status, cudaStream_t s);
+int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, const int32_t* ids, int T,
+                     const RouteWS& rw, float* Ye, int32_t* status, cudaStream_t s);
 
 static int launch_expert(const bitsmoe_plan* p, const void* blob, const float* Z, const int32_t* ids,
                          const float* gw, int T, float* Ye, float* Ysum, const RouteWS& rw, int32_t* status,
                          cudaStream_t s) {
     const int E = p->dims.n_experts, K = p->dims.top_k, d_out = p->dims.d_out;
-    int rc = launch_expert_mt(p, blob, Z, T, rw, Ye, status, s);
+    int rc = launch_expert_mt(p, blob, Z, ids, T, rw, Ye, status, s);
     if (rc) return rc;
     uint64_t n = (uint64_t)T * d_out;
     unsigned blocks = (unsigned)std::min<uint64_t>((n + 255) / 256, 4096);
@@ -144,7 +149,7 @@ static int launch_route(const bitsmoe_plan* p, const int32_t* ids, int T, const 
 
 static uint64_t expert_ws(const bitsmoe_plan* p, int T, bool need_ye, uint8_t* base, RouteWS* rw, float** ye) {
     WsCursor c{base, 0};
-    RouteWS r = take_route(c, p->dims.n_experts, T, p->dims.top_k);
+    RouteWS r = take_route(c, p->dims.n_experts, T, p->dims.top_k, cvals_ldc(p));
     float* y = need_ye ? (float*)c.take(4ull * T * p->dims.top_k * p->dims.d_out) : nullptr;
     if (rw) *rw = r;
     if (ye) *ye = y;
@@ -192,7 +197,7 @@ static uint64_t layer_ws(const bitsmoe_plan* g, const bitsmoe_plan* u, int T, co
                          uint8_t* base, LayerWS* out) {
     WsCursor c{base, 0};
     LayerWS L;
-    L.route = take_route(c, g->dims.n_experts, T, g->dims.top_k);
+    L.route = take_route(c, g->dims.n_experts, T, g->dims.top_k, std::max(cvals_ldc(g), cvals_ldc(u)));
     const bitsmoe_plan* p[2] = {g, u};
     for (int j = 0; j < 2; j++) {
         L.Z[j] = (!io || !io[j]->Z) ? (float*)c.take(4ull * T * p[j]->dims.rank) : nullptr;

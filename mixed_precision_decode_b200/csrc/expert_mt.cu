@@ -6,39 +6,43 @@
 //             - sum_b (2^b - 1)/2 sum_{k in G_b} c_{k,t}
 //             + sum_{k in G_16} a_k z_{t,k} w16_{k,i},        c_{k,t} = a_k s_k z_{t,k}.
 //
-// Design: one CTA per (routed expert, range of 32-row tiles).  The CTA stages
-// its tiles' planes and the expert's per-component metadata in shared memory
-// with a few TMA bulk copies (a run of tiles of one group is contiguous), then
-// loops over the expert's tokens in groups of four.  Per group it forms c for
-// every member and token, and per chunk of 128 members it builds 16-entry
-// subset-sum tables whose entries are token PAIRS (float2): one conflict-free
-// 8-byte shared load answers a 4-member nibble for two tokens, so the
-// bit-serial sum costs one byte-permute and two loads per nibble for four
-// tokens.  A warp owns one 32-row tile (a lane per row); when a CTA stages
-// fewer than 8 tiles, several warps share a tile and split its plane words.
+// Two kernels.  k_cvals forms, once per routed (token, slot) pair, c for every
+// member of the pair's expert (a_k z_{t,k} for the fp16 members) and the
+// pair's zero-point total, into a workspace buffer.  k_expert_mt then runs one
+// CTA per (routed expert, range of up to 4 tiles of 32 rows), 16 warps, two
+// CTAs per SM: it stages its tiles of every plane word in shared memory with
+// 16-byte cp.async pieces from every thread (a plane word gives a CTA only
+// 128 B per tile, too little for a bulk copy apiece) and the c rows of up to
+// four of the expert's tokens with one bulk copy each.  Each warp takes a contiguous
+// range of the expert's member words (balanced by plane words) and, per word,
+// builds in its own 2 KB of shared memory the word's 16-entry subset-sum
+// tables whose entries are token PAIRS (float2), with shuffles, then looks up
+// every plane word of the member word for every tile: one conflict-free 8-byte
+// shared load per 4-member nibble and two tokens, a lane per row.  The loop
+// needs no CTA barrier; the warps' partial sums are added in warp order at the
+// end, so the outputs do not depend on timing.
 #include <algorithm>
 
 #include "common.cuh"
 
 namespace bitsmoe {
 
-constexpr int kMtThreads = 256;
+constexpr int kMtThreads = 512;  // 16 warps; two CTAs share an SM
 constexpr int kMtWarps = kMtThreads / 32;
 constexpr int kMtTok = 4;           // tokens per group
 constexpr int kMtPairs = kMtTok / 2;
-constexpr int kMtCW = 4;            // 32-member words per chunk
+constexpr int kMtMaxTiles = 4;      // 32-row tiles per CTA, at most
+constexpr int kCvThreads = 256;
 constexpr long long kMtWaitNs = 2000000000LL;
 
 struct MtParams {
     const uint8_t* blob;
-    const float* Z;
     RouteWS rw;
     float* Ye;
     int32_t* status;
-    int r, K, d_out, d_pad, n_tiles;
-    int tiles_per_cta;  // 1, 2, 4 or 8 (warps per tile = 8 / tiles_per_cta)
-    uint32_t stage_words, meta_bytes, c_floats;
-    uint32_t sm_stage, sm_meta, sm_c, sm_tab, sm_misc;
+    int K, d_out, d_pad, n_tiles;
+    int tiles_per_cta;  // 1, 2 or 4
+    uint32_t sm_stage, sm_c, sm_tab;
 };
 
 __device__ __forceinline__ uint32_t mt_smem_u32(const void* p) {
@@ -51,7 +55,6 @@ __device__ __forceinline__ long long mt_globaltimer() {
 }
 __device__ __forceinline__ void mt_mbar_init(uint64_t* bar) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mt_smem_u32(bar)));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ void mt_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mt_smem_u32(bar)), "r"(bytes)
@@ -85,22 +88,82 @@ __device__ __forceinline__ float2 mt_lds2(uint32_t addr) {
 }
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
 
+// ---------------------------------------------------------------------------
+// c values: one CTA per routed pair q = t * K + j
+// ---------------------------------------------------------------------------
+// C[q][m] over the member slots m of the pair's expert, groups in storage
+// order (fp16 first), each padded to its np: a_k s_k z_{t,k} for the bit-plane
+// members, a_k z_{t,k} for the fp16 members, 0 for padding (and for an index
+// k >= r, which only a corrupt blob holds).  zp[q] = sum over the bit-plane
+// groups of (2^b - 1)/2 sum_k c_k.
+__global__ void __launch_bounds__(kCvThreads) k_cvals(const uint8_t* __restrict__ blob, const float* __restrict__ Z,
+                                                      const int32_t* __restrict__ ids, int K, int E, int r,
+                                                      RouteWS rw) {
+    __shared__ float s_red[kCvThreads / 32];
+    const int q = blockIdx.x, t = q / K, tid = threadIdx.x;
+    const int e = ids[q];
+    if (e < 0 || e >= E) return;  // the routing groups leave this pair out
+    const DirEntry d = read_dir(blob, e);
+    float* Cq = rw.cvals + (size_t)q * rw.ldc;
+    const float* zt = Z + (size_t)t * r;
+    uint32_t off = 0;
+    float zsum = 0.0f;
+    for (int g = 0; g < kNumGroups; g++) {
+        const int b = group_width(g);
+        const uint32_t n = d.count[g], np = (uint32_t)group_members_padded(b, n);
+        if (np == 0) continue;
+        const uint8_t* gm = blob + d.base + d.goff[g];
+        const uint16_t* idx = reinterpret_cast<const uint16_t*>(gm);
+        const float hr = 0.5f * (float)((1 << b) - 1);
+        for (uint32_t m = tid; m < np; m += kCvThreads) {
+            float c = 0.0f;
+            if (m < n) {
+                const int k = idx[m];
+                if (k < r) {
+                    if (b == 16) {
+                        c = reinterpret_cast<const float*>(gm + 2ull * np)[m] * __ldg(zt + k);
+                    } else {
+                        const uint16_t sh = reinterpret_cast<const uint16_t*>(gm + 2ull * np)[m];
+                        c = reinterpret_cast<const float*>(gm + 4ull * np)[m] * __half2float(__ushort_as_half(sh)) *
+                            __ldg(zt + k);
+                        zsum += hr * c;
+                    }
+                }
+            }
+            Cq[off + m] = c;
+        }
+        off += np;
+    }
+    for (int o = 16; o > 0; o >>= 1) zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
+    if ((tid & 31) == 0) s_red[tid >> 5] = zsum;
+    __syncthreads();
+    if (tid == 0) {
+        float s = 0.0f;
+        for (int w = 0; w < kCvThreads / 32; w++) s += s_red[w];
+        rw.zp[q] = s;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// expert evaluation: one CTA per (routed expert, range of tiles)
+// ---------------------------------------------------------------------------
 // Per-expert shape of the staged data.
 struct MtExpert {
     uint32_t n[kNumGroups], np[kNumGroups], W[kNumGroups];
     uint32_t stage_off[kNumGroups];  // word offset of the group's tiles in the staging buffer
-    uint32_t meta_off[kNumGroups];   // byte offset of the group's metadata in the staging buffer
-    uint32_t c_off[kNumGroups];      // member offset of the group in the c buffer (bit-plane groups)
+    uint32_t c_off[kNumGroups];      // member offset of the group in a c row
     uint64_t gbase[kNumGroups];      // byte offset of the group in the blob
-    uint32_t members;                // padded bit-plane members
+    uint32_t members;                // padded members of all groups: the length of a c row
+    uint32_t plane_words;            // b W summed over the bit-plane groups
 };
 
 __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ uint64_t s_bar;
+    __shared__ uint64_t s_cbar;  // the c rows of a token group (one phase per group)
     __shared__ MtExpert s_ex;
-    __shared__ int s_tok[kMtTok], s_pair[kMtTok], s_fail;
-    __shared__ float s_zpw[kMtWarps][kMtTok], s_zpt[kMtTok];
+    __shared__ int s_pair[kMtTok], s_fail;
+    __shared__ float s_zp[kMtTok];
+    __shared__ int s_wbeg[kMtWarps + 1];  // member words of each warp (a contiguous range)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int slot = blockIdx.x;
@@ -110,220 +173,233 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     const int tile0 = blockIdx.y * P.tiles_per_cta;
     const int ntl = min(P.tiles_per_cta, P.n_tiles - tile0);
     if (ntl <= 0) return;
-    const int wpt = kMtWarps / P.tiles_per_cta;  // warps per tile
-    const int my_tile = warp / wpt, part = warp % wpt;
-    const int row = (tile0 + my_tile) * 32 + lane;
-    const bool tile_ok = my_tile < ntl;
 
     uint32_t* s_stage = reinterpret_cast<uint32_t*>(smem + P.sm_stage);
-    uint8_t* s_meta = smem + P.sm_meta;
-    float* s_c = reinterpret_cast<float*>(smem + P.sm_c);  // [member][kMtTok]
-    // token-pair tables: 1024-byte aligned blocks of (word, pair) -> 8 nibble tables x 16 float2
+    float* s_c = reinterpret_cast<float*>(smem + P.sm_c);  // [token][members]
+    // each warp's token-pair tables: a 2048-byte block (pair 0, then pair 1) of
+    // 8 nibble tables x 16 float2, on a 1024-byte boundary
     const uint32_t tab_raw = mt_smem_u32(smem + P.sm_tab);
     const uint32_t tab_s = (tab_raw + 1023u) & ~1023u;
     float2* s_tab = reinterpret_cast<float2*>(smem + P.sm_tab + (tab_s - tab_raw));
-    float* s_red = reinterpret_cast<float*>(s_tab);  // reused after the last chunk: [warp][32][kMtTok]
+    float2* my_tab = s_tab + (size_t)warp * 256;
+    const uint32_t my_tab_s = tab_s + 2048u * (uint32_t)warp;
+    float* s_part = reinterpret_cast<float*>(s_tab);  // reused after the lookups: [warp][tile][32][kMtTok]
 
-    // ---- stage the expert's metadata and this CTA's rows of every plane word ----
+    // ---- stage this CTA's rows of every plane word of the expert ----
     if (warp == 0) {
-      if (lane == 0) {
-        const DirEntry d = read_dir(P.blob, e);
-        uint32_t so = 0, mo = 0, co = 0;
-        for (int g = 0; g < kNumGroups; g++) {
-            const int b = group_width(g);
-            s_ex.n[g] = d.count[g];
-            s_ex.np[g] = (uint32_t)group_members_padded(b, d.count[g]);
-            s_ex.W[g] = b == 16 ? 0 : s_ex.np[g] / 32;
-            s_ex.stage_off[g] = so;
-            s_ex.meta_off[g] = mo;
-            s_ex.c_off[g] = co;
-            s_ex.gbase[g] = d.base + d.goff[g];
-            if (b != 16) {
-                so += (uint32_t)ntl * b * s_ex.W[g] * 32;
+        if (lane == 0) {
+            const DirEntry d = read_dir(P.blob, e);
+            uint32_t so = 0, co = 0, pw = 0;
+            for (int g = 0; g < kNumGroups; g++) {
+                const int b = group_width(g);
+                s_ex.n[g] = d.count[g];
+                s_ex.np[g] = (uint32_t)group_members_padded(b, d.count[g]);
+                s_ex.W[g] = b == 16 ? 0 : s_ex.np[g] / 32;
+                s_ex.stage_off[g] = so;
+                s_ex.c_off[g] = co;
+                s_ex.gbase[g] = d.base + d.goff[g];
+                if (b != 16) {
+                    so += (uint32_t)ntl * b * s_ex.W[g] * 32;
+                    pw += (uint32_t)b * s_ex.W[g];
+                }
                 co += s_ex.np[g];
             }
-            mo += (b == 16 ? 6u : 8u) * s_ex.np[g];
-        }
-        s_ex.members = co;
-        s_fail = 0;
-        mt_mbar_init(&s_bar);
-        mt_expect_tx(&s_bar, 4 * so + mo);
-        for (int g = 0; g < kNumGroups; g++) {
-            if (s_ex.n[g] == 0) continue;
-            const int b = group_width(g);
-            mt_bulk(s_meta + s_ex.meta_off[g], P.blob + s_ex.gbase[g], (b == 16 ? 6u : 8u) * s_ex.np[g], &s_bar);
-        }
-      }
-      __syncwarp();
-      // plane word q of group g: rows [32 tile0, 32 (tile0 + ntl)) are contiguous in the
-      // blob ([b][W][d_pad], rows fastest) and staged as [b][W][32 ntl]
-      const uint64_t d_pad = 32ull * P.n_tiles;
-      int g = 1, qg = 0;  // group of plane word q, and its first word
-      for (int q = lane;; q += 32) {
-          while (g < kNumGroups && q >= qg + group_width(g) * (int)s_ex.W[g]) {
-              qg += group_width(g) * (int)s_ex.W[g];
-              g++;
-          }
-          if (g >= kNumGroups) break;
-          const uint8_t* planes = P.blob + s_ex.gbase[g] + 8ull * s_ex.np[g];
-          mt_bulk(s_stage + s_ex.stage_off[g] + (uint32_t)(q - qg) * 32u * ntl,
-                  planes + 4ull * ((uint64_t)(q - qg) * d_pad + 32ull * tile0), 128u * ntl, &s_bar);
-      }
-      if (lane == 0 && !mt_mbar_wait(&s_bar, 0)) {
-          s_fail = 1;
-          if (P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
-      }
-    }
-    __syncthreads();
-    if (s_fail) return;
-
-    const int myt = tid % kMtTok;  // token whose c values this thread forms
-    for (int pq = p0; pq < p1; pq += kMtTok) {
-        const int nt = min(kMtTok, p1 - pq);
-        __syncthreads();  // the previous group's outputs are written
-        if (tid < kMtTok) {
-            const int pr = tid < nt ? P.rw.pairs[pq + tid] : -1;
-            s_pair[tid] = pr;
-            s_tok[tid] = pr >= 0 ? pr / P.K : -1;
-        }
-        __syncthreads();
-        // c_{k,t} = a_k s_k z_{t,k} of every bit-plane member, and the zero-point partials
-        {
-            const int tok = s_tok[myt];
-            const float* zt = P.Z + (size_t)(tok < 0 ? 0 : tok) * P.r;
-            float zp = 0.0f;
+            s_ex.members = co;
+            // member words (in group order) shared out over the warps by plane words:
+            // warp v takes the words that start in [pw v / warps, pw (v + 1) / warps)
+            int wv = 0;
+            uint32_t acc_pw = 0, word = 0;
+            s_wbeg[0] = 0;
             for (int g = 1; g < kNumGroups; g++) {
-                const uint32_t np = s_ex.np[g], n = s_ex.n[g];
-                if (np == 0) continue;
-                const uint8_t* gm = s_meta + s_ex.meta_off[g];
-                const uint16_t* idx = reinterpret_cast<const uint16_t*>(gm);
-                const uint16_t* scl = reinterpret_cast<const uint16_t*>(gm + 2 * np);
-                const float* amp = reinterpret_cast<const float*>(gm + 4 * np);
-                const float hr = 0.5f * (float)((1 << group_width(g)) - 1);
-                float* cg = s_c + (size_t)s_ex.c_off[g] * kMtTok;
-                // four values per pass: every load of a pass is issued before its stores
-                for (uint32_t v0 = tid; v0 < np * kMtTok; v0 += 4 * kMtThreads) {
-                    float c[4];
-#pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const uint32_t v = v0 + u * kMtThreads, m = v / kMtTok;
-                        c[u] = (v < np * kMtTok && m < n && tok >= 0)
-                                   ? amp[m] * __half2float(__ushort_as_half(scl[m])) * __ldg(zt + idx[m])
-                                   : 0.0f;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const uint32_t v = v0 + u * kMtThreads;
-                        if (v < np * kMtTok) cg[v] = c[u];
-                        zp += hr * c[u];
-                    }
+                const uint32_t b = (uint32_t)group_width(g);
+                for (uint32_t w = 0; w < s_ex.W[g]; w++, word++) {
+                    while (wv < kMtWarps - 1 && (uint64_t)acc_pw * kMtWarps >= (uint64_t)pw * (wv + 1)) s_wbeg[++wv] = (int)word;
+                    acc_pw += b;
                 }
             }
-            // lanes with equal lane % kMtTok hold the same token
-            for (int o = kMtTok; o < 32; o <<= 1) zp += __shfl_xor_sync(0xffffffffu, zp, o);
-            if (lane < kMtTok) s_zpw[warp][lane] = zp;
+            while (wv < kMtWarps) s_wbeg[++wv] = (int)word;
+            s_fail = 0;
+            mt_mbar_init(&s_cbar);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            s_ex.plane_words = pw;
         }
-        __syncthreads();
-        if (tid < kMtTok) {
-            float s = 0.0f;
-            for (int w = 0; w < kMtWarps; w++) s += s_zpw[w][tid];
-            s_zpt[tid] = s;
+    }
+    __syncthreads();  // s_ex, the word ranges and the mbarriers are ready
+    // ---- stage this CTA's rows of every plane word of the expert: plane word q of
+    // group g holds rows [32 tile0, 32 (tile0 + ntl)) contiguously in the blob ([b][W][d_pad],
+    // rows fastest); they are staged as [b][W][32 ntl], by every thread in 16-byte
+    // pieces (cp.async: a CTA's plane words are too many, and each too short, for
+    // one bulk copy apiece) ----
+    {
+        const uint32_t per_word = 8u * (uint32_t)ntl;  // 16-byte pieces of one plane word's rows
+        const uint32_t total = s_ex.plane_words * per_word;
+        int g = 1;
+        uint32_t qg = 0;  // first plane word of group g
+        for (uint32_t i = tid; i < total; i += kMtThreads) {
+            const uint32_t q = i / per_word, piece = i - q * per_word;
+            while (q >= qg + (uint32_t)group_width(g) * s_ex.W[g]) {
+                qg += (uint32_t)group_width(g) * s_ex.W[g];
+                g++;
+            }
+            const uint8_t* src = P.blob + s_ex.gbase[g] + 8ull * s_ex.np[g] +
+                                 4ull * ((uint64_t)(q - qg) * (uint64_t)P.d_pad + 32ull * tile0) + 16ull * piece;
+            const uint32_t dst = mt_smem_u32(s_stage + s_ex.stage_off[g] + (q - qg) * 32u * ntl + 4u * piece);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
         }
-        float2 acc[kMtPairs];
-#pragma unroll
-        for (int q = 0; q < kMtPairs; q++) acc[q] = make_float2(0.0f, 0.0f);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const uint32_t members = s_ex.members;
+    const int wbeg = s_wbeg[warp], wend = s_wbeg[warp + 1];
 
-        for (int g = 1; g < kNumGroups; g++) {
-            const int b = group_width(g);
-            const uint32_t W = s_ex.W[g];
-            if (W == 0) continue;
-            const float* cg = s_c + (size_t)s_ex.c_off[g] * kMtTok;
-            const uint32_t* stg = s_stage + s_ex.stage_off[g];
-            for (uint32_t w0 = 0; w0 < W; w0 += kMtCW) {
-                const int cw = (int)min((uint32_t)kMtCW, W - w0);
-                __syncthreads();  // the previous chunk's tables are no longer read
-                // entry x = ((wi * kMtPairs + pair) * 8 + n) * 16 + e: sum of c over the set bits of e
-                for (int x = tid; x < cw * kMtPairs * 128; x += kMtThreads) {
-                    const int en = x & 15, n = (x >> 4) & 7, wp = x >> 7;
-                    const int pair = wp % kMtPairs, wi = wp / kMtPairs;
-                    const float* cm = cg + (size_t)(32 * (w0 + wi) + 4 * n) * kMtTok + 2 * pair;
-                    float2 v = make_float2(0.0f, 0.0f);
+    uint32_t cphase = 0;
+    for (int pq = p0; pq < p1; pq += kMtTok) {
+        const int nt = min(kMtTok, p1 - pq);
+        __syncthreads();  // the previous group's c rows and partial sums are no longer read
+        // ---- the c rows of this group's tokens (one bulk copy each) ----
+        if (tid == 0) {
+            mt_expect_tx(&s_cbar, 4u * members * (uint32_t)nt);
+            for (int u = 0; u < kMtTok; u++) {
+                const int pr = u < nt ? P.rw.pairs[pq + u] : -1;
+                s_pair[u] = pr;
+                s_zp[u] = pr >= 0 ? P.rw.zp[pr] : 0.0f;
+                if (pr >= 0 && members > 0)
+                    mt_bulk(s_c + (size_t)u * members, P.rw.cvals + (size_t)pr * P.rw.ldc, 4u * members, &s_cbar);
+            }
+            if (!mt_mbar_wait(&s_cbar, cphase)) s_fail = 1;
+        }
+        cphase ^= 1u;
+        if (pq == p0) asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's pieces of the planes
+        __syncthreads();
+        if (s_fail) {
+            if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
+            return;
+        }
+
+        // acc[tile][pair]: this warp's partial sums for its rows of every tile
+        float2 acc[kMtMaxTiles][kMtPairs];
 #pragma unroll
-                    for (int bit = 0; bit < 4; bit++)
-                        if (en & (1 << bit)) v = f2add(v, *reinterpret_cast<const float2*>(cm + bit * kMtTok));
-                    s_tab[x] = v;
+        for (int t = 0; t < kMtMaxTiles; t++)
+#pragma unroll
+            for (int q = 0; q < kMtPairs; q++) acc[t][q] = make_float2(0.0f, 0.0f);
+
+        // ---- this warp's member words, in group order: its own tables, then every
+        // plane word of the member word for every tile of the CTA ----
+        int g = 1, wg0 = 0;  // group of the current word, and its first word index
+        for (int wi = wbeg; wi < wend; wi++) {
+            while (wi >= wg0 + (int)s_ex.W[g]) {
+                wg0 += (int)s_ex.W[g];
+                g++;
+            }
+            const int b = group_width(g), w = wi - wg0;
+            const uint32_t W = s_ex.W[g];
+            const float* cg = s_c + s_ex.c_off[g];
+            const uint32_t m = 32u * (uint32_t)w + (uint32_t)lane;
+            float c[kMtTok];
+#pragma unroll
+            for (int u = 0; u < kMtTok; u++) c[u] = u < nt ? cg[(size_t)u * members + m] : 0.0f;
+            __syncwarp();  // the previous word's lookups are done with the tables
+            // entry en of table tb of pair pr = the sums of c over the set bits of en
+            // (members 4 tb .. 4 tb + 3) for tokens 2 pr and 2 pr + 1
+            const int en = lane & 15;
+#pragma unroll
+            for (int pr = 0; pr < kMtPairs; pr++) {
+#pragma unroll
+                for (int qq = 0; qq < 4; qq++) {
+                    const int tb = (lane >> 4) + 2 * qq;
+                    const float x0 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb);
+                    const float x1 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb + 1);
+                    const float x2 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb + 2);
+                    const float x3 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb + 3);
+                    const float y0 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb);
+                    const float y1 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb + 1);
+                    const float y2 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb + 2);
+                    const float y3 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb + 3);
+                    float2 v;
+                    v.x = ((en & 1 ? x0 : 0.0f) + (en & 2 ? x1 : 0.0f)) + ((en & 4 ? x2 : 0.0f) + (en & 8 ? x3 : 0.0f));
+                    v.y = ((en & 1 ? y0 : 0.0f) + (en & 2 ? y1 : 0.0f)) + ((en & 4 ? y2 : 0.0f) + (en & 8 ? y3 : 0.0f));
+                    my_tab[(pr * 8 + tb) * 16 + en] = v;
                 }
-                __syncthreads();
-                if (!tile_ok) continue;
-                for (int q = part; q < b * cw; q += wpt) {
-                    const int j = q / cw, wi = q - j * cw;
-                    const uint32_t word = stg[(((uint32_t)j * W + w0 + wi) * ntl + my_tile) * 32 + lane];
+            }
+            __syncwarp();  // the tables are written
+            const uint32_t* stg = s_stage + s_ex.stage_off[g] + (uint32_t)w * (uint32_t)ntl * 32u + (uint32_t)lane;
+            for (int j = 0; j < b; j++) {
+                const float wt = (float)(1u << j);
+                const uint32_t* sj = stg + (uint32_t)j * W * (uint32_t)ntl * 32u;
+#pragma unroll
+                for (int t = 0; t < kMtMaxTiles; t++) {
+                    if (t >= ntl) break;
+                    const uint32_t word = sj[t * 32];
                     // entry offsets (nibble x 8 bytes): even nibbles in the bytes of lo, odd in hi
                     const uint32_t lo = (word << 3) & 0x78787878u, hi = (word >> 1) & 0x78787878u;
-                    const uint32_t base = tab_s + 2048u * (uint32_t)wi;  // (wi, pair 0); pair 1 at +1024
-                    const uint32_t a0 = __byte_perm(lo, base, 0x7650u), a1 = __byte_perm(hi, base, 0x7650u);
-                    const uint32_t a2 = __byte_perm(lo, base, 0x7651u), a3 = __byte_perm(hi, base, 0x7651u);
-                    const uint32_t a4 = __byte_perm(lo, base, 0x7652u), a5 = __byte_perm(hi, base, 0x7652u);
-                    const uint32_t a6 = __byte_perm(lo, base, 0x7653u), a7 = __byte_perm(hi, base, 0x7653u);
-                    const float wt = (float)(1u << j);
+                    const uint32_t a0 = __byte_perm(lo, my_tab_s, 0x7650u), a1 = __byte_perm(hi, my_tab_s, 0x7650u);
+                    const uint32_t a2 = __byte_perm(lo, my_tab_s, 0x7651u), a3 = __byte_perm(hi, my_tab_s, 0x7651u);
+                    const uint32_t a4 = __byte_perm(lo, my_tab_s, 0x7652u), a5 = __byte_perm(hi, my_tab_s, 0x7652u);
+                    const uint32_t a6 = __byte_perm(lo, my_tab_s, 0x7653u), a7 = __byte_perm(hi, my_tab_s, 0x7653u);
                     {
                         const float2 s = f2add(f2add(f2add(mt_lds2<0>(a0), mt_lds2<128>(a1)),
                                                      f2add(mt_lds2<256>(a2), mt_lds2<384>(a3))),
                                                f2add(f2add(mt_lds2<512>(a4), mt_lds2<640>(a5)),
                                                      f2add(mt_lds2<768>(a6), mt_lds2<896>(a7))));
-                        acc[0].x = fmaf(s.x, wt, acc[0].x);
-                        acc[0].y = fmaf(s.y, wt, acc[0].y);
+                        acc[t][0].x = fmaf(s.x, wt, acc[t][0].x);
+                        acc[t][0].y = fmaf(s.y, wt, acc[t][0].y);
                     }
                     {
                         const float2 s = f2add(f2add(f2add(mt_lds2<1024>(a0), mt_lds2<1152>(a1)),
                                                      f2add(mt_lds2<1280>(a2), mt_lds2<1408>(a3))),
                                                f2add(f2add(mt_lds2<1536>(a4), mt_lds2<1664>(a5)),
                                                      f2add(mt_lds2<1792>(a6), mt_lds2<1920>(a7))));
-                        acc[1].x = fmaf(s.x, wt, acc[1].x);
-                        acc[1].y = fmaf(s.y, wt, acc[1].y);
+                        acc[t][1].x = fmaf(s.x, wt, acc[t][1].x);
+                        acc[t][1].y = fmaf(s.y, wt, acc[t][1].y);
                     }
                 }
             }
         }
-        // fp16 group: a_k z_{t,k} w16_{k,i}
-        if (s_ex.n[0] > 0 && tile_ok && row < P.d_out) {
+        // fp16 group: (a_k z_{t,k}) w16_{k,i}, rows read in place; member m to warp m % warps
+        if (s_ex.n[0] > 0) {
             const uint32_t np = s_ex.np[0];
-            const uint8_t* gm = s_meta + s_ex.meta_off[0];
-            const uint16_t* idx = reinterpret_cast<const uint16_t*>(gm);
-            const float* amp = reinterpret_cast<const float*>(gm + 2 * np);
             const uint16_t* w16 = reinterpret_cast<const uint16_t*>(P.blob + s_ex.gbase[0] + 6ull * np);
-            for (uint32_t m = part; m < s_ex.n[0]; m += wpt) {
-                const float wv = __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row]));
-                float cz[kMtTok];
+            const float* c16 = s_c + s_ex.c_off[0];
+            for (uint32_t mm = warp; mm < s_ex.n[0]; mm += kMtWarps) {
+                const float cz0 = c16[mm], cz1 = c16[members + mm], cz2 = c16[2 * members + mm],
+                            cz3 = c16[3 * members + mm];
 #pragma unroll
-                for (int t = 0; t < kMtTok; t++)
-                    cz[t] = s_tok[t] >= 0 ? amp[m] * __ldg(P.Z + (size_t)s_tok[t] * P.r + idx[m]) : 0.0f;
-                acc[0].x = fmaf(cz[0], wv, acc[0].x);
-                acc[0].y = fmaf(cz[1], wv, acc[0].y);
-                acc[1].x = fmaf(cz[2], wv, acc[1].x);
-                acc[1].y = fmaf(cz[3], wv, acc[1].y);
+                for (int t = 0; t < kMtMaxTiles; t++) {
+                    if (t >= ntl) break;
+                    const int row = (tile0 + t) * 32 + lane;
+                    const float wv = __half2float(__ushort_as_half(w16[(size_t)mm * P.d_pad + row]));
+                    acc[t][0].x = fmaf(cz0, wv, acc[t][0].x);
+                    acc[t][0].y = fmaf(cz1, wv, acc[t][0].y);
+                    acc[t][1].x = fmaf(cz2, wv, acc[t][1].x);
+                    acc[t][1].y = fmaf(cz3, wv, acc[t][1].y);
+                }
             }
         }
-        // warps sharing a tile add their partial sums; the first writes the rows
-        __syncthreads();  // tables are no longer read: s_red reuses them
-        float* red = s_red + ((size_t)warp * 32 + lane) * kMtTok;
-        red[0] = acc[0].x;
-        red[1] = acc[0].y;
-        red[2] = acc[1].x;
-        red[3] = acc[1].y;
+        // ---- the warps' partial sums, added in warp order; warp t writes tile t ----
+        __syncthreads();  // every warp is done with its tables: s_part reuses them
+#pragma unroll
+        for (int t = 0; t < kMtMaxTiles; t++) {
+            if (t >= ntl) break;
+            float* pp = s_part + (((size_t)warp * kMtMaxTiles + t) * 32 + lane) * kMtTok;
+            pp[0] = acc[t][0].x;
+            pp[1] = acc[t][0].y;
+            pp[2] = acc[t][1].x;
+            pp[3] = acc[t][1].y;
+        }
         __syncthreads();
-        if (part == 0 && tile_ok && row < P.d_out) {
+        for (int t = warp; t < ntl; t += kMtWarps) {
+            const int row = (tile0 + t) * 32 + lane;
+            if (row >= P.d_out) continue;
             float y[kMtTok];
 #pragma unroll
-            for (int t = 0; t < kMtTok; t++) y[t] = -s_zpt[t];
-            for (int w = warp; w < warp + wpt; w++) {
-                const float* rr = s_red + ((size_t)w * 32 + lane) * kMtTok;
+            for (int u = 0; u < kMtTok; u++) y[u] = -s_zp[u];
+            for (int v = 0; v < kMtWarps; v++) {
+                const float* pp = s_part + (((size_t)v * kMtMaxTiles + t) * 32 + lane) * kMtTok;
 #pragma unroll
-                for (int t = 0; t < kMtTok; t++) y[t] += rr[t];
+                for (int u = 0; u < kMtTok; u++) y[u] += pp[u];
             }
 #pragma unroll
-            for (int t = 0; t < kMtTok; t++)
-                if (t < nt) P.Ye[(size_t)s_pair[t] * P.d_out + row] = y[t];
+            for (int u = 0; u < kMtTok; u++)
+                if (u < nt) P.Ye[(size_t)s_pair[u] * P.d_out + row] = y[u];
         }
     }
 }
@@ -333,67 +409,67 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
 // ---------------------------------------------------------------------------
 static int g_mt_max_smem = 0;
 
-int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, int T, const RouteWS& rw, float* Ye,
-                     int32_t* status, cudaStream_t s) {
+// Floats per c row: every expert's padded members, rounded to 8 (32-byte rows).
+uint32_t cvals_ldc(const bitsmoe_plan* p) { return (uint32_t)roundup(p->max_members_padded, 8); }
+
+int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, const int32_t* ids, int T,
+                     const RouteWS& rw, float* Ye, int32_t* status, cudaStream_t s) {
     if (g_mt_max_smem == 0) {
         int dev;
         cudaError_t e = cudaGetDevice(&dev);
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_mt_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return set_cuda_error(e);
     }
+    if (rw.ldc < cvals_ldc(p)) return BITSMOE_EINVAL;
+    const int npairs = T * p->dims.top_k;
+    k_cvals<<<(unsigned)npairs, kCvThreads, 0, s>>>((const uint8_t*)blob, Z, ids, p->dims.top_k, p->dims.n_experts,
+                                                    p->dims.rank, rw);
+    int rc = check_launch();
+    if (rc) return rc;
+
     MtParams P{};
     P.blob = (const uint8_t*)blob;
-    P.Z = Z;
     P.rw = rw;
     P.Ye = Ye;
     P.status = status;
-    P.r = p->dims.rank;
     P.K = p->dims.top_k;
     P.d_out = p->dims.d_out;
     P.d_pad = (int)p->d_pad;
     P.n_tiles = (int)(p->d_pad / 32);
-    // per-expert maxima: words of one tile over the bit-plane groups, metadata bytes, members
-    uint64_t tile_words = 0, meta = 0, members = 0;
+    // per-expert maximum of the words of one tile over the bit-plane groups
+    uint64_t tile_words = 0;
     for (int e = 0; e < p->dims.n_experts; e++) {
         const uint32_t* c = p->counts + 8 * (size_t)e;
-        uint64_t tw = 0, mb = 0, mm = 0;
+        uint64_t tw = 0;
         for (int g = 0; g < kNumGroups; g++) {
             const int b = group_width(g);
-            const uint64_t np = group_members_padded(b, c[g]);
-            mb += (b == 16 ? 6 : 8) * np;
-            if (b != 16) {
-                tw += (uint64_t)b * (np / 32) * 32;
-                mm += np;
-            }
+            if (b != 16) tw += (uint64_t)b * (group_members_padded(b, c[g]) / 32) * 32;
         }
         tile_words = std::max(tile_words, tw);
-        meta = std::max(meta, mb);
-        members = std::max(members, mm);
     }
-    const uint64_t fixed = roundup(meta, 128) + roundup(members * kMtTok * 4, 128) + 8192 + 1024 + 128;
+    // c rows of kMtTok tokens, and each warp's tables (2 KB, + 1024 for their
+    // alignment), which the warps' partial sums reuse at the end
+    static_assert(kMtWarps * kMtMaxTiles * 32 * kMtTok * 4 <= kMtWarps * 2048, "partial sums fit the tables");
+    const uint64_t fixed = roundup(4ull * kMtTok * p->max_members_padded, 128) + kMtWarps * 2048ull + 1024 + 128;
     const uint64_t budget = (uint64_t)g_mt_max_smem - 1024;  // static shared memory of the kernel
-    // the most tiles per CTA that still lets two CTAs share an SM (more warps hide the
-    // shared-memory latency of the lookups); else the most that fit one CTA per SM
+    // the most tiles per CTA that still lets two CTAs share an SM (one stages while
+    // the other computes); else the most that fit one CTA per SM
     const uint64_t half = (uint64_t)g_mt_max_smem / 2 - 1024;
-    int tpc = 8;
+    int tpc = kMtMaxTiles;
     while (tpc > 1 && fixed + 4 * tile_words * tpc > half) tpc /= 2;
     if (fixed + 4 * tile_words * tpc > half) {
-        tpc = 8;
+        tpc = kMtMaxTiles;
         while (tpc > 1 && fixed + 4 * tile_words * tpc > budget) tpc /= 2;
     }
     if (fixed + 4 * tile_words * tpc > budget) return BITSMOE_ESIZE;  // one tile does not fit
     P.tiles_per_cta = tpc;
-    P.stage_words = (uint32_t)(tile_words * tpc);
-    P.meta_bytes = (uint32_t)roundup(meta, 128);
-    P.c_floats = (uint32_t)(members * kMtTok);
     P.sm_stage = 0;
-    P.sm_meta = (uint32_t)roundup(4ull * P.stage_words, 128);
-    P.sm_c = P.sm_meta + P.meta_bytes;
-    P.sm_tab = (uint32_t)(P.sm_c + roundup(4ull * P.c_floats, 128));
-    const size_t smem = P.sm_tab + 8192 + 1024;
+    P.sm_c = (uint32_t)roundup(4ull * tile_words * tpc, 128);
+    P.sm_tab = P.sm_c + (uint32_t)roundup(4ull * kMtTok * p->max_members_padded, 128);
+    const size_t smem = P.sm_tab + kMtWarps * 2048 + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_expert_mt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return set_cuda_error(e);
-    const int slots = (int)std::min<int64_t>((int64_t)p->dims.n_experts, (int64_t)T * P.K);
+    const int slots = (int)std::min<int64_t>((int64_t)p->dims.n_experts, (int64_t)npairs);
     dim3 grid((unsigned)slots, (unsigned)((P.n_tiles + tpc - 1) / tpc));
     k_expert_mt<<<grid, kMtThreads, smem, s>>>(P);
     return check_launch();
