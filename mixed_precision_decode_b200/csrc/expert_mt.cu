@@ -32,6 +32,7 @@ constexpr int kMtWarps = kMtThreads / 32;
 constexpr int kMtTok = 4;           // tokens per group
 constexpr int kMtPairs = kMtTok / 2;
 constexpr int kMtMaxTiles = 4;      // 32-row tiles per CTA, at most
+constexpr uint32_t kMtBuildCost = 5;  // a member word's table build, in lookups of one plane word, tile and pair
 constexpr int kCvThreads = 256;
 constexpr long long kMtWaitNs = 2000000000LL;
 
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     if (warp == 0) {
         if (lane == 0) {
             const DirEntry d = read_dir(P.blob, e);
-            uint32_t so = 0, co = 0, pw = 0;
+            uint32_t so = 0, co = 0, pw = 0, pwords = 0;
             for (int g = 0; g < kNumGroups; g++) {
                 const int b = group_width(g);
                 s_ex.n[g] = d.count[g];
@@ -200,13 +201,15 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                 s_ex.gbase[g] = d.base + d.goff[g];
                 if (b != 16) {
                     so += (uint32_t)ntl * b * s_ex.W[g] * 32;
-                    pw += (uint32_t)b * s_ex.W[g];
+                    pw += (uint32_t)s_ex.W[g] * (2u * (uint32_t)b * (uint32_t)ntl + kMtBuildCost);
+                    pwords += (uint32_t)b * s_ex.W[g];
                 }
                 co += s_ex.np[g];
             }
             s_ex.members = co;
-            // member words (in group order) shared out over the warps by plane words:
-            // warp v takes the words that start in [pw v / warps, pw (v + 1) / warps)
+            // member words (in group order) shared out over the warps by cost (the
+            // lookups of b planes x ntl tiles x 2 token pairs, plus one table build):
+            // warp v takes the words whose cost starts in [pw v / warps, pw (v + 1) / warps)
             int wv = 0;
             uint32_t acc_pw = 0, word = 0;
             s_wbeg[0] = 0;
@@ -214,14 +217,14 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                 const uint32_t b = (uint32_t)group_width(g);
                 for (uint32_t w = 0; w < s_ex.W[g]; w++, word++) {
                     while (wv < kMtWarps - 1 && (uint64_t)acc_pw * kMtWarps >= (uint64_t)pw * (wv + 1)) s_wbeg[++wv] = (int)word;
-                    acc_pw += b;
+                    acc_pw += 2u * b * (uint32_t)ntl + kMtBuildCost;
                 }
             }
             while (wv < kMtWarps) s_wbeg[++wv] = (int)word;
             s_fail = 0;
             mt_mbar_init(&s_cbar);
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            s_ex.plane_words = pw;
+            s_ex.plane_words = pwords;
         }
     }
     __syncthreads();  // s_ex, the word ranges and the mbarriers are ready
@@ -237,10 +240,11 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
         uint32_t qg = 0;  // first plane word of group g
         for (uint32_t i = tid; i < total; i += kMtThreads) {
             const uint32_t q = i / per_word, piece = i - q * per_word;
-            while (q >= qg + (uint32_t)group_width(g) * s_ex.W[g]) {
+            while (g < kNumGroups && q >= qg + (uint32_t)group_width(g) * s_ex.W[g]) {
                 qg += (uint32_t)group_width(g) * s_ex.W[g];
                 g++;
             }
+            if (g >= kNumGroups) break;  // only past the expert's plane words (never, if the counts agree)
             const uint8_t* src = P.blob + s_ex.gbase[g] + 8ull * s_ex.np[g] +
                                  4ull * ((uint64_t)(q - qg) * (uint64_t)P.d_pad + 32ull * tile0) + 16ull * piece;
             const uint32_t dst = mt_smem_u32(s_stage + s_ex.stage_off[g] + (q - qg) * 32u * ntl + 4u * piece);
@@ -254,6 +258,7 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     uint32_t cphase = 0;
     for (int pq = p0; pq < p1; pq += kMtTok) {
         const int nt = min(kMtTok, p1 - pq);
+        const int npairs = (nt + 1) / 2;  // token pairs with a routed token (the second is skipped if empty)
         __syncthreads();  // the previous group's c rows and partial sums are no longer read
         // ---- the c rows of this group's tokens (one bulk copy each) ----
         if (tid == 0) {
@@ -286,7 +291,7 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
         // plane word of the member word for every tile of the CTA ----
         int g = 1, wg0 = 0;  // group of the current word, and its first word index
         for (int wi = wbeg; wi < wend; wi++) {
-            while (wi >= wg0 + (int)s_ex.W[g]) {
+            while (g < kNumGroups - 1 && wi >= wg0 + (int)s_ex.W[g]) {
                 wg0 += (int)s_ex.W[g];
                 g++;
             }
@@ -303,6 +308,7 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
             const int en = lane & 15;
 #pragma unroll
             for (int pr = 0; pr < kMtPairs; pr++) {
+                if (pr >= npairs) break;
 #pragma unroll
                 for (int qq = 0; qq < 4; qq++) {
                     const int tb = (lane >> 4) + 2 * qq;
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                         acc[t][0].x = fmaf(s.x, wt, acc[t][0].x);
                         acc[t][0].y = fmaf(s.y, wt, acc[t][0].y);
                     }
-                    {
+                    if (npairs > 1) {
                         const float2 s = f2add(f2add(f2add(mt_lds2<1024>(a0), mt_lds2<1152>(a1)),
                                                      f2add(mt_lds2<1280>(a2), mt_lds2<1408>(a3))),
                                                f2add(f2add(mt_lds2<1536>(a4), mt_lds2<1664>(a5)),
