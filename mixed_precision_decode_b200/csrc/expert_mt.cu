@@ -33,7 +33,8 @@ constexpr int kMtTok = 4;           // tokens per group
 constexpr int kMtPairs = kMtTok / 2;
 constexpr int kMtMaxTiles = 4;      // 32-row tiles per CTA, at most
 constexpr uint32_t kMtBuildCost = 5;  // a member word's table build, in lookups of one plane word, tile and pair
-constexpr int kCvThreads = 256;
+constexpr int kCvThreads = 1024;
+constexpr int kCvPer = 2;          // members of a c row per thread and pass
 constexpr long long kMtWaitNs = 2000000000LL;
 
 struct MtParams {
@@ -101,47 +102,66 @@ __global__ void __launch_bounds__(kCvThreads) k_cvals(const uint8_t* __restrict_
                                                       const int32_t* __restrict__ ids, int K, int E, int r,
                                                       RouteWS rw) {
     __shared__ float s_red[kCvThreads / 32];
+    __shared__ uint32_t start[kNumGroups + 1], s_n[kNumGroups];  // first c slot and members of each group
+    __shared__ const uint8_t* s_gm[kNumGroups];                  // each group's metadata
     const int q = blockIdx.x, t = q / K, tid = threadIdx.x;
     const int e = ids[q];
     if (e < 0 || e >= E) return;  // the routing groups leave this pair out
-    const DirEntry d = read_dir(blob, e);
+    if (tid == 0) {
+        const DirEntry d = read_dir(blob, e);
+        start[0] = 0;
+        for (int g = 0; g < kNumGroups; g++) {
+            start[g + 1] = start[g] + (uint32_t)group_members_padded(group_width(g), d.count[g]);
+            s_n[g] = d.count[g];
+            s_gm[g] = blob + d.base + d.goff[g];
+        }
+    }
+    __syncthreads();
     float* Cq = rw.cvals + (size_t)q * rw.ldc;
     const float* zt = Z + (size_t)t * r;
-    uint32_t off = 0;
     float zsum = 0.0f;
-    for (int g = 0; g < kNumGroups; g++) {
-        const int b = group_width(g);
-        const uint32_t n = d.count[g], np = (uint32_t)group_members_padded(b, n);
-        if (np == 0) continue;
-        const uint8_t* gm = blob + d.base + d.goff[g];
-        const uint16_t* idx = reinterpret_cast<const uint16_t*>(gm);
-        const float hr = 0.5f * (float)((1 << b) - 1);
-        for (uint32_t m = tid; m < np; m += kCvThreads) {
-            float c = 0.0f;
-            if (m < n) {
-                const int k = idx[m];
-                if (k < r) {
-                    if (b == 16) {
-                        c = reinterpret_cast<const float*>(gm + 2ull * np)[m] * __ldg(zt + k);
+    // kCvPer members a thread per pass; every load of a pass is issued before its z loads
+    for (uint32_t m0 = 0; m0 < start[kNumGroups]; m0 += kCvThreads * kCvPer) {
+        int kk[kCvPer], gg[kCvPer];
+        float f[kCvPer];  // a_k s_k (bit-plane member) or a_k (fp16 member); 0 for padding
+#pragma unroll
+        for (int v = 0; v < kCvPer; v++) {
+            const uint32_t m = m0 + (uint32_t)tid + (uint32_t)v * kCvThreads;
+            int g = 0;
+#pragma unroll
+            for (int h = 1; h < kNumGroups; h++) g += m >= start[h] ? 1 : 0;
+            gg[v] = m < start[kNumGroups] ? g : -1;
+            kk[v] = r;
+            f[v] = 0.0f;
+            if (gg[v] >= 0) {
+                const uint32_t ml = m - start[g], np = start[g + 1] - start[g];
+                if (ml < s_n[g]) {
+                    const uint8_t* gm = s_gm[g];
+                    kk[v] = reinterpret_cast<const uint16_t*>(gm)[ml];
+                    if (group_width(g) == 16) {
+                        f[v] = reinterpret_cast<const float*>(gm + 2ull * np)[ml];
                     } else {
-                        const uint16_t sh = reinterpret_cast<const uint16_t*>(gm + 2ull * np)[m];
-                        c = reinterpret_cast<const float*>(gm + 4ull * np)[m] * __half2float(__ushort_as_half(sh)) *
-                            __ldg(zt + k);
-                        zsum += hr * c;
+                        const uint16_t sh = reinterpret_cast<const uint16_t*>(gm + 2ull * np)[ml];
+                        f[v] = reinterpret_cast<const float*>(gm + 4ull * np)[ml] * __half2float(__ushort_as_half(sh));
                     }
                 }
             }
-            Cq[off + m] = c;
         }
-        off += np;
+#pragma unroll
+        for (int v = 0; v < kCvPer; v++) {
+            if (gg[v] < 0) continue;
+            const float c = kk[v] < r ? f[v] * __ldg(zt + kk[v]) : 0.0f;
+            Cq[m0 + (uint32_t)tid + (uint32_t)v * kCvThreads] = c;
+            if (gg[v] > 0) zsum += 0.5f * (float)((1 << group_width(gg[v])) - 1) * c;
+        }
     }
     for (int o = 16; o > 0; o >>= 1) zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
     if ((tid & 31) == 0) s_red[tid >> 5] = zsum;
     __syncthreads();
     if (tid == 0) {
-        float s = 0.0f;
-        for (int w = 0; w < kCvThreads / 32; w++) s += s_red[w];
-        rw.zp[q] = s;
+        float sum = 0.0f;
+        for (int w = 0; w < kCvThreads / 32; w++) sum += s_red[w];
+        rw.zp[q] = sum;
     }
 }
 
