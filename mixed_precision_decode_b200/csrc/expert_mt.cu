@@ -89,6 +89,13 @@ __device__ __forceinline__ float2 mt_lds2(uint32_t addr) {
     return v;
 }
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+// 4-byte shared load (one token) at a 32-bit shared address plus a constant.
+template <int OFF>
+__device__ __forceinline__ float mt_lds1(uint32_t addr) {
+    float v;
+    asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
+    return v;
+}
 
 // ---------------------------------------------------------------------------
 // c values: one CTA per routed pair q = t * K + j
@@ -323,6 +330,42 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
 #pragma unroll
             for (int u = 0; u < kMtTok; u++) c[u] = u < nt ? cg[(size_t)u * members + m] : 0.0f;
             __syncwarp();  // the previous word's lookups are done with the tables
+            if (nt == 1) {
+                // one token: float tables (8 x 16 entries, 512 B), one 4-byte lookup per
+                // nibble -- half the shared-memory traffic of a token pair
+                float* tab1 = reinterpret_cast<float*>(my_tab);
+                const int e1 = lane & 15;
+#pragma unroll
+                for (int qq = 0; qq < 4; qq++) {
+                    const int tb = (lane >> 4) + 2 * qq;
+                    const float x0 = __shfl_sync(0xffffffffu, c[0], 4 * tb);
+                    const float x1 = __shfl_sync(0xffffffffu, c[0], 4 * tb + 1);
+                    const float x2 = __shfl_sync(0xffffffffu, c[0], 4 * tb + 2);
+                    const float x3 = __shfl_sync(0xffffffffu, c[0], 4 * tb + 3);
+                    tab1[tb * 16 + e1] =
+                        ((e1 & 1 ? x0 : 0.0f) + (e1 & 2 ? x1 : 0.0f)) + ((e1 & 4 ? x2 : 0.0f) + (e1 & 8 ? x3 : 0.0f));
+                }
+                __syncwarp();
+                const uint32_t* stg1 = s_stage + s_ex.stage_off[g] + (uint32_t)w * (uint32_t)ntl * 32u + (uint32_t)lane;
+                for (int j = 0; j < b; j++) {
+                    const float wt = (float)(1u << j);
+                    const uint32_t* sj = stg1 + (uint32_t)j * W * (uint32_t)ntl * 32u;
+#pragma unroll
+                    for (int t = 0; t < kMtMaxTiles; t++) {
+                        if (t >= ntl) break;
+                        const uint32_t word = sj[t * 32];
+                        // entry offsets (nibble x 4 bytes): even nibbles in the bytes of lo, odd in hi
+                        const uint32_t lo = (word << 2) & 0x3C3C3C3Cu, hi = (word >> 2) & 0x3C3C3C3Cu;
+                        const float sum =
+                            ((mt_lds1<0>(__byte_perm(lo, my_tab_s, 0x7650u)) + mt_lds1<64>(__byte_perm(hi, my_tab_s, 0x7650u))) +
+                             (mt_lds1<128>(__byte_perm(lo, my_tab_s, 0x7651u)) + mt_lds1<192>(__byte_perm(hi, my_tab_s, 0x7651u)))) +
+                            ((mt_lds1<256>(__byte_perm(lo, my_tab_s, 0x7652u)) + mt_lds1<320>(__byte_perm(hi, my_tab_s, 0x7652u))) +
+                             (mt_lds1<384>(__byte_perm(lo, my_tab_s, 0x7653u)) + mt_lds1<448>(__byte_perm(hi, my_tab_s, 0x7653u))));
+                        acc[t][0].x = fmaf(sum, wt, acc[t][0].x);
+                    }
+                }
+                continue;
+            }
             // entry en of table tb of pair pr = the sums of c over the set bits of en
             // (members 4 tb .. 4 tb + 3) for tokens 2 pr and 2 pr + 1
             const int en = lane & 15;

@@ -13,16 +13,20 @@ namespace bitsmoe {
 
 constexpr int kSPWarps = 8;
 
+// acc + the products of 8 fp16 pairs: mixed-precision FMAs (fp16 operands, exact
+// in fp32; fp32 addend), no fp16 value converted on its own.
 __device__ __forceinline__ float dot8(uint4 a, uint4 b, float acc) {
-    const __half2* ha = reinterpret_cast<const __half2*>(&a);
-    const __half2* hb = reinterpret_cast<const __half2*>(&b);
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-        float2 fa = __half22float2(ha[j]);
-        float2 fb = __half22float2(hb[j]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
-    }
+    asm("{\n"
+        " .reg .f16 a0, a1, a2, a3, a4, a5, a6, a7, b0, b1, b2, b3, b4, b5, b6, b7;\n"
+        " mov.b32 {a0, a1}, %1;\n mov.b32 {a2, a3}, %2;\n mov.b32 {a4, a5}, %3;\n mov.b32 {a6, a7}, %4;\n"
+        " mov.b32 {b0, b1}, %5;\n mov.b32 {b2, b3}, %6;\n mov.b32 {b4, b5}, %7;\n mov.b32 {b6, b7}, %8;\n"
+        " fma.rn.f32.f16 %0, a0, b0, %0;\n fma.rn.f32.f16 %0, a1, b1, %0;\n"
+        " fma.rn.f32.f16 %0, a2, b2, %0;\n fma.rn.f32.f16 %0, a3, b3, %0;\n"
+        " fma.rn.f32.f16 %0, a4, b4, %0;\n fma.rn.f32.f16 %0, a5, b5, %0;\n"
+        " fma.rn.f32.f16 %0, a6, b6, %0;\n fma.rn.f32.f16 %0, a7, b7, %0;\n"
+        "}"
+        : "+f"(acc)
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
     return acc;
 }
 
