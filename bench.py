@@ -109,6 +109,35 @@ def algorithmic_bytes(cfg, counts, ids_step, T) -> dict:
             "distinct_experts": int(len(experts))}
 
 
+def lds_wavefronts(cfg, counts, ids_step, T) -> int:
+    """Shared-memory wavefronts (128 B each) of the multi-token expert kernel's
+    table lookups for one layer step.  Per distinct routed expert and token group
+    of up to 4 of its tokens, every plane word (bit planes of 32 members, padded)
+    is looked up in every 32-row tile: one 4-byte lookup per 4 bits (8 wavefronts
+    per warp) for a one-token group, else two 8-byte lookups per 4 bits for each
+    token pair (16 wavefronts per pair)."""
+    import numpy as np
+    tiles = (cfg.d_out + 31) // 32
+    ids = ids_step.reshape(-1)
+    experts, per_expert = np.unique(ids, return_counts=True)
+    widths = (8, 6, 4, 3, 2, 1)  # the bit-plane groups, storage order after fp16
+    total = 0
+    for proj in ("gate", "up"):
+        c = counts[proj]
+        for e, te in zip(experts, per_expert):
+            n = c[int(e)]
+            pw = sum(b * ((int(n[g + 1]) + 31) // 32) for g, b in enumerate(widths))
+            groups = [4] * (int(te) // 4) + ([int(te) % 4] if int(te) % 4 else [])
+            per_tile = sum(8 if nt == 1 else 16 * ((nt + 1) // 2) for nt in groups)
+            total += pw * tiles * per_tile
+    return total
+
+
+def lds_peak_gbs(sm_mhz: float, sms: int = 148) -> float:
+    """Shared-memory bandwidth from the unit counts: 128 B per clock per SM."""
+    return 128.0 * sms * sm_mhz * 1e6 / 1e9
+
+
 def plan_counts(plan) -> "np.ndarray":
     import numpy as np
     h = plan.header()
@@ -365,6 +394,9 @@ def run_ours(args, dist):
     # algorithmic bytes per step, averaged over the steps in the graph
     bys = [algorithmic_bytes(cfg, wl.counts[wl.layer_of(s)], wl.ids[s].cpu().numpy(), T) for s in range(G)]
     alg = {k: float(np.mean([b[k] for b in bys])) for k in bys[0]}
+    # shared-memory wavefronts of the multi-token expert lookups per step (T > 1)
+    lds_wf = float(np.mean([lds_wavefronts(cfg, wl.counts[wl.layer_of(s)], wl.ids[s].cpu().numpy(), T)
+                            for s in range(G)])) if T > 1 else 0.0
 
     # warm-up (eager), then capture G steps into a graph (and the remainder).  The
     # steps run as a decode loop: each call names the layer that runs next (it
@@ -440,6 +472,15 @@ def run_ours(args, dist):
         "clocks": clocks.summary(),
         "e2e": e2e,
     }
+    if T > 1:
+        # the expert lookups' own bound: shared-memory wavefronts over the whole step's time
+        # (a lower bound on the kernel's rate), against 128 B per clock per SM at the sampled clock
+        lds_peak = lds_peak_gbs(line["clocks"].get("sm_mhz") or 1965.0, torch.cuda.get_device_properties(0).multi_processor_count)
+        lds_achieved = lds_wf * 128 / step_s / 1e9
+        line["roofline_lds"] = {"bound": "lds", "kernel": "k_expert_mt (table lookups, both projections)",
+                                "achieved": lds_achieved, "peak": lds_peak, "peak_kind": "unit counts x sampled SM clock",
+                                "unit": "GB/s", "frac": lds_achieved / lds_peak,
+                                "wavefronts_per_step": lds_wf, "duration_us": step_s * 1e6}
     if ms_chained is not None:
         value_ch, step_ch = weak_scaling_throughput(dist.world, K, T, ms_chained)
         line["chained"] = {"value": value_ch, "ms_per_step": step_ch * 1e3,
