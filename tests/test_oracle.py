@@ -179,7 +179,7 @@ def test_quantiser_b1_is_sign(orc):
 def test_quantiser_is_nearest_level(orc, b):
     """Brute force over all 2^b levels in fp64: q picks the nearest level (ties up).
     Cases within 1e-5 relative of a tie are skipped: there fp32 rounding of p/s
-    decides, as specified, and fp64 cannot serve as the judge."""
+    decides, as specified, and fp64 cannot settle it."""
     rng = np.random.default_rng(b)
     levels_q = np.arange(2 ** b)
     for _ in range(40):
