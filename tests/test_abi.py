@@ -126,3 +126,26 @@ def test_chained_call_rejects_one_next_pointer(B):
     assert rc == B.EINVAL
     rc = L.bitsmoe_layer_forward_chained(None, None, None, None, None, 1, None, 0, 256, 264, None, None)
     assert rc == B.EINVAL
+
+
+def test_workspace_holds_the_multi_token_c_rows(B):
+    """The expert and layer workspaces hold, per routed pair, a c row as long as the
+    largest expert's padded member list (rounded up to 8 floats), its zero-point
+    total and its output row."""
+    rng = np.random.default_rng(7)
+    E, r, d_out, K = 5, 100, 40, 2
+    w = _widths(rng, E, r)
+    plan = B.pack_plan(8, d_out, E, r, K, w)
+
+    def padded(b, n):
+        return 0 if n == 0 else (-(-n // 8) * 8 if b == 16 else -(-n // 32) * 32)
+
+    members = max(sum(padded(int(b), int((w[e] == b).sum())) for b in (16, 8, 6, 4, 3, 2, 1)) for e in range(E))
+    ldc = -(-members // 8) * 8
+    for T in (1, 3, 17):
+        per_pair = 4 * ldc + 4 + 4 * d_out
+        assert B.expert_workspace_bytes(plan, T) >= T * K * per_pair
+        assert B.layer_workspace_bytes(plan, plan, T) >= T * K * (4 * ldc + 4)
+    # each buffer is rounded up to 256 bytes: the growth may fall short by that per buffer
+    grow = B.expert_workspace_bytes(plan, 17) - B.expert_workspace_bytes(plan, 3)
+    assert grow >= 14 * K * per_pair - 3 * 256
