@@ -264,8 +264,6 @@ struct Item {
 };
 // A member word (32 members of a group) whose c values and tables this CTA builds.
 struct MemberWord {
-    const uint8_t* meta;  // the group's metadata: idx u16[np] | scale fp16[np] | amp f32[np]
-    uint32_t np;          // padded members of the group
     int16_t p, g, w;
     int16_t nvalid;  // real members in the word (0..32)
     int16_t zp;      // 1 when this CTA evaluates the word's plane 0 and so owns its zero-point share
@@ -502,8 +500,6 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         if (newmw) {
             const UnitInfo& U = s_unit[my_u];
             MemberWord M;
-            M.meta = P.proj[U.p].blob + U.gbase[g];
-            M.np = U.np[g];
             M.p = (int16_t)U.p;
             M.g = (int16_t)g;
             M.w = (int16_t)w;
