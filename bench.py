@@ -312,6 +312,48 @@ def cores_used() -> int:
     return 1  # the oracle is single-threaded C
 
 
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def time_oracle_threads(sample, threads: int, seconds: float) -> tuple[float, int]:
+    """The oracle on `threads` host threads at once, each running whole layer steps
+    (its C calls release the interpreter lock; it keeps no mutable global state):
+    elapsed seconds and steps completed."""
+    import threading
+    counts = [0] * threads
+    deadline = time.perf_counter() + seconds
+
+    def work(k):
+        i = k
+        while time.perf_counter() < deadline:
+            sample.run(i)
+            counts[k] += 1
+            i += threads
+
+    ts = [threading.Thread(target=work, args=(k,)) for k in range(threads)]
+    t0 = time.perf_counter()
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    return time.perf_counter() - t0, sum(counts)
+
+
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
@@ -493,6 +535,12 @@ def run_ours(args, dist):
         line["cpu_baseline"] = {"value": n * T / el, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
                                 "sample": f"{n} full layer steps ({len(samp.items)} distinct pre-packed steps of "
                                           f"layer 0, packing untimed), {el:.1f} s, single-threaded C oracle"}
+        # the same oracle on every host core: independent layer steps on one thread per core
+        nthr = host_cores()
+        el_a, n_a = time_oracle_threads(samp, nthr, args.cpu_seconds)
+        line["cpu_baseline"]["all_cores"] = {
+            "value": n_a * T / el_a, "unit": "tokens/s", "cores": nthr, "cpu": cpu_model(),
+            "sample": f"{n_a} full layer steps on {nthr} threads (one per core, each its own steps), {el_a:.1f} s"}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 

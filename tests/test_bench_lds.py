@@ -44,3 +44,29 @@ def test_every_width_group_counts_its_planes():
 
 def test_lds_peak_from_unit_counts():
     assert abs(bench.lds_peak_gbs(1965.0, 148) - 128 * 148 * 1.965) < 1e-6
+
+
+class _TinyOracleStep:
+    """A layer step of the real oracle on tiny inputs (Phi^T x for 4 rows)."""
+
+    def __init__(self):
+        import oracle
+        oracle.build()
+        self.o = oracle
+        rng = np.random.default_rng(3)
+        self.phi = rng.standard_normal((4, 64)).astype(np.float16).view(np.uint16)
+        self.x = rng.standard_normal((1, 64)).astype(np.float16).view(np.uint16)
+        self.ref = self.o.shared_proj(self.phi, self.x)
+        self.bad = 0
+
+    def run(self, i):
+        z = self.o.shared_proj(self.phi, self.x)
+        if not np.array_equal(z, self.ref):
+            self.bad += 1
+
+
+def test_oracle_on_every_host_core_runs_independent_steps():
+    s = _TinyOracleStep()
+    el, n = bench.time_oracle_threads(s, 3, 0.3)
+    assert el >= 0.3 and n >= 3 and s.bad == 0
+    assert bench.host_cores() >= 1 and isinstance(bench.cpu_model(), str)
