@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-chained", action="store_true", help="skip the chained-loop measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--clock-window", type=float, default=0.25,
+                    help="seconds of untimed replays of the same loop before the timed steps, during which (and "
+                         "during the timed steps) the SM clock is sampled")
     return ap.parse_args()
 
 
@@ -190,12 +193,17 @@ class Workload:
     def layer_of(self, s):
         return s % len(self.layers)
 
+    def data_of(self, s):
+        return s % self.n_steps
+
     def step(self, s, stream=None, next_s=None):
-        """Step s; with next_s, as a decode loop that runs step next_s after it
-        (its layer's Phi^T is prefetched while this step evaluates experts)."""
-        l = self.layer_of(s)
+        """Step s of the decode loop (any integer): layer s mod L on pre-drawn
+        token and routing s mod n_steps.  With next_s, as a decode loop that runs
+        step next_s after it (its layer's Phi^T is prefetched while this step
+        evaluates experts)."""
+        l, d = self.layer_of(s), self.data_of(s)
         nxt = None if next_s is None else self.layers[self.layer_of(next_s)]
-        self.layers[l].forward(self.x[s], self.ids[s], self.gw[s], out=self.out[l], stream=stream, next_layer=nxt)
+        self.layers[l].forward(self.x[d], self.ids[d], self.gw[d], out=self.out[l], stream=stream, next_layer=nxt)
 
     def blob_bytes_total(self):
         return sum(L.gate.blob.numel() + L.up.blob.numel() + 2 * L.gate.phi_t.numel() * 2 for L in self.layers) // 2 * 2
@@ -205,33 +213,74 @@ class Workload:
 # clocks during the timed region (NVML reads only)
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event reasons from NVML (reads only; no GPU setting is
+    changed).  A thread polls while the sampler is entered; `sample_now()` adds
+    one sample from the calling thread.  With `timed_events` = (ev0, ev1) set,
+    the poll thread spins without sleeping while ev0 has completed and ev1 has
+    not, and counts those samples as taken inside the timed region."""
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.ok = False
+        self.period = period_s
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h = self._handle(pynvml, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._get_r = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
             self.ok = True
         except Exception as e:  # no NVML: report that instead of clocks
             self.err = str(e)
-        self.samples, self.reasons = [], 0
+        self.samples, self.timed_samples, self.reasons = [], [], 0
+        self.timed_events = None
+        self._lock = threading.Lock()
         self._stop = threading.Event()
 
+    @staticmethod
+    def _handle(nv, index: int):
+        """NVML handle of CUDA device `index`, matched by UUID (NVML numbers every GPU
+        of the host; CUDA only the visible ones), else by index."""
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(index).uuid)
+            u = u if u.startswith("GPU-") else "GPU-" + u
+            return nv.nvmlDeviceGetHandleByUUID(u)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(index)
+
+    def sample_now(self, in_timed: bool = False):
+        if not self.ok:
+            return
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            r = int(self._get_r(self.h))
+        except Exception:
+            return
+        with self._lock:
+            self.samples.append(mhz)
+            if in_timed:
+                self.timed_samples.append(mhz)
+            self.reasons |= r
+
+    def _in_timed(self) -> bool:
+        ev = self.timed_events
+        if ev is None:
+            return False
+        try:
+            return bool(ev[0].query()) and not bool(ev[1].query())
+        except Exception:
+            return False
+
     def _run(self):
-        nv = self.nv
-        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                self.reasons |= int(get_r(self.h))
-            except Exception:
-                pass
-            time.sleep(0.002)
+            inside = self._in_timed()
+            self.sample_now(inside)
+            if not inside:
+                time.sleep(self.period)
 
     def __enter__(self):
         if self.ok:
@@ -250,40 +299,55 @@ class ClockSampler:
         import statistics
         names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+                "reasons": names, "samples": len(self.samples), "samples_in_timed_region": len(self.timed_samples),
+                "sm_mhz_in_timed_region": statistics.median(self.timed_samples) if self.timed_samples else None}
 
 
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
-class OracleSample:
-    """Pre-packed oracle inputs for a few steps of layer 0 (packing untimed)."""
+def oracle_sample_steps(n_steps: int, n_layers: int, want: int = 4) -> list[int]:
+    """Steps of layer 0 (step s runs layer s mod n_layers) that the workload holds,
+    at most `want` of them and never none: the oracle baseline runs layer 0's
+    factors on those steps' tokens and routing."""
+    n_layers = max(1, n_layers)
+    steps = list(range(0, max(1, n_steps), n_layers))[:max(1, want)]
+    return steps or [0]
 
-    def __init__(self, wl: Workload, steps, frac: float = 1.0):
+
+class OracleSample:
+    """Pre-packed oracle inputs for a few layer steps (packing untimed).
+
+    factors: {"gate"|"up": {"phi_t", "amps", "comps", "widths"}} as torch tensors
+    (any device; only the routed experts are copied to the host); steps: a list
+    of (x [T][d_in] fp16, ids [T][top_k] int32, gate_w [T][top_k] f32) tensors.
+    Uses synth's tensors and the oracle only: no part of the CUDA library."""
+
+    def __init__(self, factors: dict, steps: list, rank: int, frac: float = 1.0):
         import numpy as np
+        import torch
         import oracle
         oracle.build()
         self.o = oracle
-        cfg = wl.cfg
-        self.r_sub = max(1, int(round(frac * cfg.rank)))
-        self.frac = self.r_sub / cfg.rank
-        h = wl.host0
+        self.r_sub = max(1, int(round(frac * rank)))
+        self.frac = self.r_sub / rank
         self.items = []
-        for s in steps:
-            ids = wl.ids[s].cpu().numpy()
-            g = wl.gw[s].cpu().numpy()
-            x = wl.x[s].cpu().numpy().view(np.uint16)
+        for x_t, ids_t, g_t in steps:
+            ids = ids_t.cpu().numpy()
+            g = g_t.cpu().numpy()
+            x = x_t.cpu().numpy().view(np.uint16)
             ex = sorted(set(int(v) for v in ids.ravel()))
             remap = np.vectorize({e: j for j, e in enumerate(ex)}.get)(ids).astype(np.int32)
             per = {}
             for name in ("gate", "up"):
-                sel = __import__("torch").as_tensor(ex, device=h[name]["comps"].device)
-                comps = h[name]["comps"][sel][:, :self.r_sub].cpu().numpy()
-                w = h[name]["widths"][sel][:, :self.r_sub].cpu().numpy()
-                a = h[name]["amps"][sel][:, :self.r_sub].cpu().numpy()
+                h = factors[name]
+                sel = torch.as_tensor(ex, device=h["comps"].device)
+                comps = h["comps"][sel][:, :self.r_sub].cpu().numpy()
+                w = h["widths"][sel][:, :self.r_sub].cpu().numpy()
+                a = h["amps"][sel][:, :self.r_sub].cpu().numpy()
                 sc, _ = oracle.compute_scales(comps, w)
                 blob, _ = oracle.pack(comps, w, sc, a)
-                phi = h[name]["phi_t"][:self.r_sub].cpu().numpy().view(np.uint16)
+                phi = h["phi_t"][:self.r_sub].cpu().numpy().view(np.uint16)
                 per[name] = (blob, phi)
             self.items.append((x, remap, g, per))
 
@@ -399,14 +463,15 @@ def measured_traffic(config_name: str):
         return None
 
 
-def workload_config(cfg, T, n_layers, wl_bytes, touched):
+def workload_config(cfg, T, n_layers):
+    """The workload's description, the same for both arms (nothing measured in it)."""
     return {"workload": f"{cfg.name}: spectral MoE gate/up layer, Qwen3-30B-A3B-shaped" if cfg.name.startswith("qwen")
             else cfg.name,
             "d_in": cfg.d_in, "d_out": cfg.d_out, "experts": cfg.n_experts, "top_k": cfg.top_k, "rank": cfg.rank,
             "tokens_per_step": T, "widths": "8:2% 4:8% 3:20% 2:40% 1:20% 0:10% (~2.08 bits)"
             if cfg.name in ("qwen_t1", "qwen_stack") else str(cfg.width_fracs),
-            "l2": f"inputs larger than L2: {n_layers} distinct layers rotated ({wl_bytes / 1e9:.2f} GB resident), "
-                  f"{touched / 1e6:.1f} MB touched per step",
+            "l2": f"inputs larger than L2: {n_layers} distinct seeded layer copies rotated, each step its own "
+                  f"token and routing",
             "routing": cfg.routing}
 
 
@@ -427,50 +492,82 @@ def run_ours(args, dist):
         cfg = synth.scaled(cfg, tokens=args.tokens)
     T = cfg.tokens
     K, W = args.steps, args.warmup
-    G = min(K, args.graph_steps)
-    n_steps_data = max(G, args.layers)
+    G = max(1, min(K, args.graph_steps))
+    L = args.layers
+    n_steps_data = max(G, L)
     want_cpu = dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline
     wl = Workload(cfg, args.layers, n_steps_data, seed_base=10_000 + 1000 * dist.rank, keep_comps_of_layer0=want_cpu)
     stream = torch.cuda.current_stream()
 
-    # algorithmic bytes per step, averaged over the steps in the graph
-    bys = [algorithmic_bytes(cfg, wl.counts[wl.layer_of(s)], wl.ids[s].cpu().numpy(), T) for s in range(G)]
-    alg = {k: float(np.mean([b[k] for b in bys])) for k in bys[0]}
+    # algorithmic bytes per step, averaged over the K timed steps (step s: layer s mod L, data s mod n)
+    pairs = {}
+    for s in range(K):
+        key = (wl.layer_of(s), wl.data_of(s))
+        pairs[key] = pairs.get(key, 0) + 1
+    bys = {key: algorithmic_bytes(cfg, wl.counts[key[0]], wl.ids[key[1]].cpu().numpy(), T) for key in pairs}
+    alg = {k: float(sum(bys[key][k] * n for key, n in pairs.items()) / K) for k in next(iter(bys.values()))}
     # shared-memory wavefronts of the multi-token expert lookups per step (T > 1)
-    lds_wf = float(np.mean([lds_wavefronts(cfg, wl.counts[wl.layer_of(s)], wl.ids[s].cpu().numpy(), T)
-                            for s in range(G)])) if T > 1 else 0.0
+    lds_wf = float(sum(lds_wavefronts(cfg, wl.counts[key[0]], wl.ids[key[1]].cpu().numpy(), T) * n
+                       for key, n in pairs.items()) / K) if T > 1 else 0.0
 
-    # warm-up (eager), then capture G steps into a graph (and the remainder).  The
-    # steps run as a decode loop: each call names the layer that runs next (it
-    # wraps at the end of a graph, where the next replay starts again at step 0).
+    # Steps run as a decode loop over a continuing rotation: timed step s (0..K-1)
+    # is layer s mod L, and the K steps are captured in graphs of up to G steps
+    # that continue the rotation.  Before them, an untimed graph of one whole
+    # rotation (steps -L..-1) ends on layer L-1, so the first timed step's layer
+    # was last read L steps earlier (L x the step's bytes, several times L2).
+    # Each call names the step that runs next (the chained loop prefetches it).
+    side = torch.cuda.Stream()
+
+    def capture_range(start, n, chained):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for s in range(start, start + n):
+                wl.step(s, next_s=(s + 1) if chained else None)
+        return g
+
     def capture(chained):
-        for s in range(W):
-            wl.step(s % G, next_s=((s + 1) % G) if chained else None)
+        for s in range(-W - L, -L):  # eager warm-up, W steps
+            wl.step(s, next_s=(s + 1) if chained else None)
         torch.cuda.synchronize()
-        gs = []
-        for n in ([G] * (K // G)) + ([K % G] if K % G else []):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=torch.cuda.Stream()):
-                for s in range(n):
-                    wl.step(s, next_s=((s + 1) % n) if chained else None)
-            gs.append(g)
+        pre = capture_range(-L, L, chained)
+        gs = [capture_range(i, min(G, K - i), chained) for i in range(0, K, G)]
+        pre.replay()
         for g in gs[:2]:
             g.replay()
         torch.cuda.synchronize()
-        return gs
+        return pre, gs
 
-    def timed(gs, clocks=None, nvtx=False):
+    def preload_replays(pre, seconds):
+        """Replays of the one-rotation graph that keep the GPU under this same load
+        for about `seconds` (untimed; clocks are sampled meanwhile)."""
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            pre.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t = max(1e-6, e0.elapsed_time(e1) / 3e3)
+        return int(min(5000, max(2, math.ceil(seconds / t))))
+
+    def timed(pre, gs, clocks=None, nvtx=False, n_pre=0):
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         dist.barrier()
         torch.cuda.synchronize()
         if clocks:
+            clocks.timed_events = (ev0, ev1)
             clocks.__enter__()
+        for _ in range(n_pre):  # untimed: the same steps, so the clocks are read under this load
+            pre.replay()
+        if clocks:
+            clocks.sample_now()
         if nvtx:
             torch.cuda.nvtx.range_push("timed")
         ev0.record(stream)
         for g in gs:
             g.replay()
         ev1.record(stream)
+        if clocks:
+            clocks.sample_now()
         torch.cuda.synchronize()
         if nvtx:
             torch.cuda.nvtx.range_pop()
@@ -482,12 +579,14 @@ def run_ours(args, dist):
     # the same loop as a chained decode loop (next layer's Phi^T prefetched into L2), reported beside
     ms_chained = None
     if not args.no_chained:
-        graphs = capture(True)
-        ms_chained = timed(graphs)
-        del graphs
-    graphs = capture(False)
-    clocks = ClockSampler(torch.cuda.current_device())
-    ms = timed(graphs, clocks, nvtx=True)
+        pre, graphs = capture(True)
+        ms_chained = timed(pre, graphs, n_pre=1)
+        del pre, graphs
+    pre, graphs = capture(False)
+    n_pre = preload_replays(pre, args.clock_window)
+    clocks = ClockSampler(torch.cuda.current_device(), period_s=0.0)
+    ms = timed(pre, graphs, clocks, nvtx=True, n_pre=n_pre)
+    del pre, graphs
     value, step_s = weak_scaling_throughput(dist.world, K, T, ms)
 
     peak, peak_kind = load_peak()
@@ -503,7 +602,9 @@ def run_ours(args, dist):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": K, "warmup": W,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded random factors of the layer's shape; no checkpoint)",
-        "config": workload_config(cfg, T, args.layers, wl.blob_bytes_total(), alg["total"]),
+        "config": workload_config(cfg, T, args.layers),
+        "workload_bytes": {"resident_gb": wl.blob_bytes_total() / 1e9, "mb_per_step": alg["total"] / 1e6,
+                           "distinct_experts_per_step": alg["distinct_experts"]},
         "roofline": {"bound": "hbm", "kernel": dominant_kernel(launches_per_step), "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": measured_traffic(cfg.name) if launches_per_step == 1 and T == 1 else None,
@@ -511,7 +612,8 @@ def run_ours(args, dist):
                                                                                        ("phi", "planes", "meta", "act")},
                      "duration_us": step_s * 1e6},
         "gpu_launches": launches_per_step * K,
-        "clocks": clocks.summary(),
+        "clocks": dict(clocks.summary(), window=f"sampled over {n_pre} untimed replays of one rotation ({n_pre * L} "
+                                                    f"steps of the same loop) and the timed region right after them"),
         "e2e": e2e,
     }
     if T > 1:
@@ -530,7 +632,8 @@ def run_ours(args, dist):
                            "how": "the same graph-replayed loop through bitsmoe_layer_forward_chained: each call "
                                   "prefetches the next step's layer Phi^T into L2 while it evaluates experts"}
     if want_cpu:
-        samp = OracleSample(wl, [0 if args.layers == 1 else s for s in range(0, 4 * args.layers, args.layers)][:4])
+        steps = [(wl.x[d], wl.ids[d], wl.gw[d]) for d in oracle_sample_steps(wl.n_steps, L)]
+        samp = OracleSample(wl.host0, steps, cfg.rank)
         el, n = time_oracle(samp, None, args.cpu_seconds)
         line["cpu_baseline"] = {"value": n * T / el, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
                                 "sample": f"{n} full layer steps ({len(samp.items)} distinct pre-packed steps of "
@@ -607,10 +710,29 @@ def run_e2e(wl, cfg, T, n, dist):
                    "SpectralMoELayer.forward on views of it, one D2H of both Y_sum; CUDA events on the stream"}
 
 
+def host_workload(cfg, seed: int, n_steps: int) -> tuple[dict, list]:
+    """Layer-0-style factors of both projections and n_steps (x, ids, gate_w),
+    drawn by synth on the CPU: the same shapes and distributions as the GPU
+    workload, from CPU generators (so not the same values).  No part of the
+    CUDA library is used."""
+    import torch
+    from mixed_precision_decode_b200 import synth
+    cpu = torch.device("cpu")
+    gen = synth.make_generator(seed, cpu)
+    factors = {name: synth.make_projection(cfg, gen, cpu) for name in ("gate", "up")}
+    gen = synth.make_generator(seed + 999_983, cpu)
+    steps = []
+    for _ in range(n_steps):
+        x = torch.randn((cfg.tokens, cfg.d_in), generator=gen).to(torch.float16)
+        ids, gw = synth.make_routing(cfg, gen, cpu, cfg.tokens)
+        steps.append((x, ids, gw))
+    return factors, steps
+
+
 def run_reference(args, dist):
     """The oracle (plain single-threaded C, fp64) on the host cores, timed per
-    step on a bounded sample of the same workload."""
-    import torch
+    step on a bounded sample of the same workload.  Rank 0 only; the inputs come
+    from synth and the oracle alone (the CUDA library is never loaded)."""
     from mixed_precision_decode_b200 import synth
 
     if dist.rank != 0:
@@ -620,16 +742,15 @@ def run_reference(args, dist):
         cfg = synth.scaled(cfg, tokens=args.tokens)
     T = cfg.tokens
     K, W = args.steps, args.warmup
-    wl = Workload(cfg, 1, 8, seed_base=10_000, keep_comps_of_layer0=True)
-    probe = OracleSample(wl, [0], 1.0)
+    factors, steps = host_workload(cfg, 10_000, 4)
+    probe = OracleSample(factors, steps[:1], cfg.rank, 1.0)
     t0 = time.perf_counter()
     probe.run(0)
     t_full = time.perf_counter() - t0
     budget = 150.0  # seconds of timed oracle work for the whole run
     frac = min(1.0, budget / max(1e-9, (K + W) * t_full))
-    samp = OracleSample(wl, list(range(4)), frac)
-    del wl
-    torch.cuda.empty_cache()
+    samp = OracleSample(factors, steps, cfg.rank, frac)
+    del factors
     for i in range(W):
         samp.run(i)
     el, n = time_oracle(samp, K, None)
@@ -638,11 +759,12 @@ def run_reference(args, dist):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": K,
         "warmup": W, "ms_per_step": el / n * 1e3 / samp.frac, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded random factors of the layer's shape)",
-        "config": workload_config(cfg, T, 1, 0, 0),
+        "config": workload_config(cfg, T, args.layers),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+                         "cpu": cpu_model(),
                          "sample": f"each step: {samp.r_sub} of {cfg.rank} spectral components (fraction "
                                    f"{samp.frac:.4f}) of a full layer step, both projections; value scaled by "
-                                   f"1/fraction; 4 distinct pre-packed steps (packing untimed)"},
+                                   f"1/fraction; 4 distinct pre-packed steps drawn on the CPU (packing untimed)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

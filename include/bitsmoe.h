@@ -23,9 +23,12 @@
  *
  * Conventions for every call:
  *   - Pointers marked "dev" are device pointers (cudaMalloc, torch tensors...),
- *     "host" are host pointers.  The caller allocates and owns every buffer;
- *     the library never allocates device memory and keeps no device state.
- *     Plans are host objects the library allocates and bitsmoe_plan_free frees.
+ *     "host" are host pointers.  The caller allocates and owns every buffer,
+ *     and the library never allocates device memory.  The one piece of device
+ *     state it keeps is the fixed scratch array of
+ *     bitsmoe_layer_forward_t1_noalloc (static device memory of the loaded
+ *     library, used by that call only).  Plans are host objects the library
+ *     allocates and bitsmoe_plan_free frees.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every device
  *     call is asynchronous on that stream; only bitsmoe_read_status waits.
  *   - Return 0 on success or a negative BITSMOE_E* code.  Argument errors are

@@ -115,7 +115,7 @@ static int orc_width_ok(int b) {
 static uint64_t orc_roundup(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
 
 /* Bytes of one group of width b holding n members, rows padded to d_pad
- * (a multiple of 32: the planes are stored in 32-row tiles). */
+ * (a multiple of 32; the planes are stored rows fastest, [b][W][d_pad]). */
 static uint64_t orc_group_bytes(int b, uint64_t n, uint64_t d_pad) {
     if (n == 0) return 0;
     if (b == 16) {
