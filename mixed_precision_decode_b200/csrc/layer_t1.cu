@@ -42,10 +42,18 @@ constexpr int kRB = 32;           // rows per tile (one per lane)
 constexpr int kMaxUnits = 32;     // routed (projection, slot) pairs: 2 * top_k
 constexpr int kMaxItems = 32;     // work items per CTA (one planning lane each)
 constexpr int kF16Item = 8;       // fp16 members per item
-constexpr int kStageWarps = 1;    // warps that issue the plane and metadata copies
-constexpr int kPhiBars = 4;       // mbarriers over the Phi slice
+constexpr int kPhiBars = 4;       // mbarriers over the Phi slice (0 also carries x)
+constexpr int kDirBar = kPhiBars;        // the expert directories
+constexpr int kPlaneBar = kPhiBars + 1;  // the staged plane words
+constexpr int kTagBar = kPhiBars + 2;    // hands this launch's tag to the other warps
+constexpr int kPlanBar = kPhiBars + 3;   // the plan is written (the planning warp arrives)
+constexpr int kZeroBar = kPhiBars + 4;   // the zeroing warps' stores are done (each arrives)
+constexpr int kZBar = kPhiBars + 5;      // the z warps' partial rows are written (each arrives)
+constexpr int kCopyBar = kPhiBars + 6;   // the planning warp has issued the plane copies
+constexpr int kNumBars = kPhiBars + 7;
+constexpr int kMaxRowsPerCta = 32;       // z rows of one CTA: one multi-row warp reduction
+constexpr int kZWarps = 8;     // warps that compute the z rows (split along d_in)
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded waits: 2 s, then BITSMOE_ST_TIMEOUT
-constexpr int kTagBar = kPhiBars + 3;  // mbarrier that hands this launch's tag to the row warps
 constexpr int kMaxZeroCtas = 16;       // CTAs that zero the outputs (each publishes a tag)
 constexpr int kZeroSliceFloats = 16384;  // outputs zeroed per zeroing CTA, at least
 // workspace head: [0] launch counter, [1 .. kMaxZeroCtas] the zeroing CTAs' tags
@@ -74,7 +82,7 @@ struct T1Params {
     int n_zero;     // CTAs that zero the outputs (1 .. kMaxZeroCtas)
     int items_max;  // work items per CTA (upper bound over every routing)
     // dynamic shared-memory layout (byte offsets)
-    uint32_t sm_x, sm_dir, sm_phi, sm_planes, sm_mw, sm_f16, sm_c16, sm_tab, sm_end;
+    uint32_t sm_dir, sm_phi, sm_planes, sm_meta, sm_c16, sm_tab, sm_end;
 };
 
 // ---------------------------------------------------------------------------
@@ -115,6 +123,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
         if (globaltimer() - t0 > kWaitLimitNs) return false;
     return true;
 }
+// Bounded wait on an mbarrier phase with a short sleep between polls, for waiters
+// off the critical path; false on timeout.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+        __nanosleep(128);
+    }
+    return true;
+}
 // Bulk copy global -> shared with an L2 cache policy (createpolicy).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
     asm volatile(
@@ -134,14 +153,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
-}
-// Named barrier `ID` over n threads (whole warps).  The callers come out of code
-// whose trip counts differ between lanes, so the warp is reconverged first:
-// bar.sync wants all 32 lanes to execute it together.
-template <int ID>
-__device__ __forceinline__ void named_barrier(int n) {
-    __syncwarp();
-    asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(n) : "memory");
 }
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -203,88 +214,95 @@ __device__ __forceinline__ float z_poll(const unsigned long long* w, uint32_t ta
 // ---------------------------------------------------------------------------
 // routed units and the column partition
 // ---------------------------------------------------------------------------
-// One routed (projection, slot) pair.
-struct UnitInfo {
-    int p, j, e;  // projection, slot, expert (-1 when the id is out of range)
-    float g;      // gate weight
-    int pw;       // plane words
-    int n16;      // fp16 members
-    int items;    // plane words + octets of fp16 members
-    uint32_t np[kNumGroups], n[kNumGroups], pw0[kNumGroups];
-    uint64_t gbase[kNumGroups];  // byte offset of each group in the blob
+// One routed (projection, slot) pair, as the phases after the plan need it.
+struct UnitRef {
+    int p, j;  // projection, slot
+    float g;   // gate weight
 };
 
-__device__ inline void unit_info(const T1Params& P, int u, int e, const uint8_t* s_dir, UnitInfo& U) {
-    U.p = u / P.K;
-    U.j = u % P.K;
-    U.e = (e >= 0 && e < P.E) ? e : -1;
-    U.g = P.gw[U.j];
-    U.pw = U.n16 = U.items = 0;
-    for (int g = 0; g < kNumGroups; g++) {
-        U.np[g] = U.n[g] = U.pw0[g] = 0;
-        U.gbase[g] = 0;
-    }
-    if (U.e < 0) return;
-    const DirEntry d = parse_dir(s_dir + ((size_t)U.p * P.E + U.e) * kDirEntryBytes);
-    uint32_t pw = 0;
-    for (int g = 0; g < kNumGroups; g++) {
-        const int b = group_width(g);
-        U.n[g] = d.count[g];
-        U.np[g] = (uint32_t)group_members_padded(b, d.count[g]);
-        U.pw0[g] = pw;
-        U.gbase[g] = d.base + d.goff[g];
-        if (b != 16) pw += (uint32_t)b * (U.np[g] / 32);
-    }
-    U.pw = (int)pw;
-    U.n16 = (int)U.n[0];
-    U.items = U.pw + (U.n16 + kF16Item - 1) / kF16Item;
-}
+// One routed unit's layout, in the planning lane's registers: the groups of its
+// expert (storage order; all zero when the id is out of range).
+struct UnitRegs {
+    uint64_t gbase[kNumGroups];  // byte offset of each group in the blob
+    uint32_t n[kNumGroups], np[kNumGroups], pw0[kNumGroups];  // members, padded members, first plane word
+    int pw;     // plane words
+    int items;  // plane words + octets of fp16 members
+};
 
-// Plane word q of a unit -> (group, bit plane, word).  Words are ordered by
-// group, then plane, then word.
-__device__ __forceinline__ void decode_pw(const UnitInfo& U, int q, int& g, int& jb, int& w) {
-    g = 1;
+// d: the unit's directory entry in shared memory, or null for an id out of range.
+__device__ __forceinline__ void unit_regs(const uint8_t* d, UnitRegs& R) {
+    uint64_t base = 0;
+    uint32_t goff[kNumGroups], cnt[kNumGroups];
+    if (d) {
+        base = *reinterpret_cast<const uint64_t*>(d);
+        const uint32_t* go = reinterpret_cast<const uint32_t*>(d + 16);
+        const uint16_t* ct = reinterpret_cast<const uint16_t*>(d + 44);
 #pragma unroll
-    for (int gg = 2; gg < kNumGroups; gg++)
-        if ((uint32_t)q >= U.pw0[gg] && U.np[gg] > 0) g = gg;
-    const int W = (int)(U.np[g] / 32);
-    const int rel = q - (int)U.pw0[g];
-    jb = rel / W;
-    w = rel - jb * W;
+        for (int g = 0; g < kNumGroups; g++) {
+            goff[g] = go[g];
+            cnt[g] = ct[g];
+        }
+    } else {
+#pragma unroll
+        for (int g = 0; g < kNumGroups; g++) goff[g] = cnt[g] = 0;
+    }
+    uint32_t pw = 0;
+#pragma unroll
+    for (int g = 0; g < kNumGroups; g++) {
+        R.n[g] = cnt[g];
+        R.np[g] = cnt[g] == 0 ? 0u : (g == 0 ? (cnt[g] + 7u) & ~7u : (cnt[g] + 31u) & ~31u);
+        R.pw0[g] = pw;
+        R.gbase[g] = base + goff[g];
+        if (g > 0) pw += (uint32_t)group_width(g) * (R.np[g] >> 5);
+    }
+    R.pw = (int)pw;
+    R.items = R.pw + (int)((R.n[0] + kF16Item - 1) / kF16Item);
 }
 
-// One work item of a CTA: a plane word (all rows of one bit plane of 32
-// members) or an octet of fp16 members (all rows).
-struct Item {
-    const uint8_t* ptr;  // plane word: its d_pad words (one per row); octet: member row 8f
-    int16_t nf;          // octet: fp16 members in it (1..8); plane word: 0
-    int16_t slot;        // member-word slot (plane word) or octet slot
-    int16_t w;           // octet: f
-    int16_t u;           // unit
+// A unit's items, in order: the plane words of its bit-plane groups (group by
+// group in storage order; inside a group, word l = jb * W + w is bit plane jb
+// of member word w, W words per plane), then the octets of its fp16 members.
+// Every CTA takes an equal contiguous share of the concatenation over the
+// routed units.  A piece is the part of one group (or of the fp16 octets) of
+// one unit that falls in the share: items [l0, l1) of the group, which are
+// contiguous both in the blob (planes are [b][W][d_pad], rows fastest) and in
+// the CTA's item slots, so one bulk copy stages a piece's plane words.  Its
+// member words are the cyclic interval (wstart + k) mod W, k < nw, with
+// nw = min(W, l1 - l0): each gets one table slot.
+struct Piece {
+    const uint8_t* gptr;  // the group's first byte in the blob
+    uint32_t np, n;       // padded and stored members of the group
+    int16_t u, g;         // unit; group (1..6: bit planes, 0: fp16 octets)
+    int16_t l0, l1;       // items [l0, l1) of the group
+    int16_t slot0;        // the CTA's item slot of l0
+    int16_t tslot0;       // first table slot (bit-plane pieces)
+    int16_t nw, wstart;   // member words covered
+    int16_t W;            // words per plane (bit-plane pieces)
+    int16_t pad_;
 };
 // A member word (32 members of a group) whose c values and tables this CTA builds.
 struct MemberWord {
-    int16_t p, g, w;
-    int16_t nvalid;  // real members in the word (0..32)
-    int16_t zp;      // 1 when this CTA evaluates the word's plane 0 and so owns its zero-point share
-    int16_t seg;
-};
-// Consecutive plane-word items of one group: contiguous in the blob (planes
-// are [b][W][d_pad], rows fastest), so one bulk copy stages all of them.
-struct Run {
-    const uint8_t* ptr;  // the first item's words
-    int a, len;          // first item slot, items
-};
-// Consecutive member-word slots of one group with consecutive words: their idx,
-// scale and amp are each one contiguous block in the blob and in shared memory.
-struct MetaRun {
-    const uint8_t* meta;  // the group's metadata
+    const uint8_t* gptr;  // the group's first byte: idx u16[np] | scale u16[np] | amp f32[np] | planes
     uint32_t np;          // padded members of the group
-    int w, slot, len;     // first word, first slot, words
+    int16_t p, g, w;
+    int16_t nvalid;  // stored members in the word (0..32)
+    int16_t zp;      // 1 when this CTA evaluates the word's plane 0 and so owns its zero-point share
+    int16_t pad_;
 };
-// Items of one unit inside a CTA's share: plane words [i0, ip), fp16 octets [ip, i1).
+// An octet of fp16 members (idx u16[np] | amp f32[np] | w16[np][d_pad]); its
+// rows are read in place during the lookups.
+struct Octet {
+    const uint8_t* gptr;  // the fp16 group's first byte
+    uint32_t np;          // padded members of the group
+    int16_t l;            // octet index: members 8 l .. 8 l + nf - 1
+    int16_t nf;           // stored members in the octet (1..8); 0 for a plane-word item
+    int16_t u;
+    int16_t pad_;
+};
+// The items of one unit inside the CTA's share: plane words [i0, ip), fp16
+// octets [ip, i1); its member words are table slots [t0, t1).
 struct Seg {
-    int u, i0, ip, i1;
+    int u, i0, ip, i1, t0, t1;
 };
 
 // acc0 += the products of the low halves of the four fp16 pairs of a and b,
@@ -313,20 +331,52 @@ __host__ __device__ __forceinline__ int share_begin(int c, int Q, int G) {
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+// acc + (low or high fp16 of a) * (the same half of b): a mixed-precision FMA
+// (fp16 operands, exact product in fp32, fp32 addend).
+template <int HI>
+__device__ __forceinline__ float fma_f16x2(uint32_t a, uint32_t b, float acc) {
+    float r;
+    if (HI)
+        asm("{\n .reg .f16 al, ah, bl, bh;\n mov.b32 {al, ah}, %1;\n mov.b32 {bl, bh}, %2;\n"
+            " fma.rn.f32.f16 %0, ah, bh, %3;\n}" : "=f"(r) : "r"(a), "r"(b), "f"(acc));
+    else
+        asm("{\n .reg .f16 al, ah, bl, bh;\n mov.b32 {al, ah}, %1;\n mov.b32 {bl, bh}, %2;\n"
+            " fma.rn.f32.f16 %0, al, bl, %3;\n}" : "=f"(r) : "r"(a), "r"(b), "f"(acc));
+    return r;
+}
+
+// Sums v[i] over the 32 lanes for 8 rows i at once: afterwards every lane l holds
+// the sum of row l & 7 (7 halving shuffles, then 2 that add the lane groups).
+__device__ __forceinline__ float warp_sum_rows8(float (&v)[8], int lane) {
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; i++) {
+            const float send = up ? v[i] : v[i + off];
+            const float keep = up ? v[i + off] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    float r = v[0];
+    r += __shfl_xor_sync(0xffffffffu, r, 8);
+    r += __shfl_xor_sync(0xffffffffu, r, 16);
+    return r;
+}
+
 __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t s_bar[kPhiBars + 4];  // Phi chunks, the expert directories, planes, metadata, tag
-    __shared__ Run s_run[kMaxItems];
-    __shared__ MetaRun s_mrun[kMaxItems];
-    __shared__ UnitInfo s_unit[kMaxUnits];
-    __shared__ Item s_item[kMaxItems];
+    __shared__ uint64_t s_bar[kNumBars];
+    __shared__ UnitRef s_unit[kMaxUnits];
+    __shared__ Piece s_piece[kMaxItems];
     __shared__ MemberWord s_mw[kMaxItems];
-    __shared__ Seg s_seg[kMaxItems];
-    __shared__ uint2 s_desc[kMaxItems];  // plane word: (tables' shared address, 2^j bits)
+    __shared__ Octet s_oct[kMaxItems];
+    __shared__ Seg s_seg[kMaxUnits];
+    __shared__ uint2 s_desc[kMaxItems];  // plane word: (its tables' shared address, 2^jb bits)
     __shared__ float s_zpmw[kMaxItems];
-    __shared__ int s_ni, s_nmw, s_nseg, s_nrun, s_nmrun, s_abort, s_bad;
+    __shared__ float s_zpart[kZWarps][32];
+    __shared__ int s_ni, s_nmw, s_nseg, s_abort, s_bad;
     __shared__ volatile int s_zto;  // a z poll timed out
-    __shared__ uint32_t s_stage_bytes, s_meta_bytes;
     __shared__ uint32_t s_tag;      // this launch's tag (1 .. 2^32 - 1)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -335,17 +385,20 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     const int row0 = share_begin(cta, 2 * P.r, P.G), row1 = share_begin(cta + 1, 2 * P.r, P.G);
     const int nrows = row1 - row0;
     const uint32_t row_bytes = (uint32_t)P.d_in * 2;
+    // warp roles: 1 plans; 2 .. 2 + nzw - 1 compute the z rows; 0 and the rest zero the outputs
+    const int nzw = min(kZWarps, nwarps - 2);
+    const bool z_warp = warp >= 2 && warp < 2 + nzw;
+    const bool zero_warp = warp != 1 && !z_warp;
+    const int n_zero_warps = nwarps - 1 - nzw;
 
-    uint16_t* s_x = reinterpret_cast<uint16_t*>(smem + P.sm_x);
     uint8_t* s_dir = smem + P.sm_dir;  // [projection][expert] directory entries
     uint8_t* s_phi = smem + P.sm_phi;
     uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + P.sm_planes);  // [item slot][d_pad]
-    // member-word metadata, one array each, 32 members per slot
-    uint16_t* s_midx = reinterpret_cast<uint16_t*>(smem + P.sm_mw);
+    float* s_c16 = reinterpret_cast<float*>(smem + P.sm_c16);               // [item slot][8]: c of octet members
+    // member-word metadata by table slot, 32 members each: idx u16, scale u16, amp f32
+    uint16_t* s_midx = reinterpret_cast<uint16_t*>(smem + P.sm_meta);
     uint16_t* s_mscl = s_midx + 32 * P.items_max;
     float* s_mamp = reinterpret_cast<float*>(s_mscl + 32 * P.items_max);
-    uint8_t* s_f16d = smem + P.sm_f16;  // [octet]: idx u16[8] | amp f32[8]
-    float* s_c16 = reinterpret_cast<float*>(smem + P.sm_c16);  // [octet][8]
     // tables start on a 512-byte shared-memory boundary: one member word's 8
     // tables are 512 B, so the byte address of a word's tables has a zero low
     // byte and a lookup can splice the entry offset into it with one byte permute
@@ -353,33 +406,29 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     float* s_tab = reinterpret_cast<float*>(tab_raw + ((512u - (smem_u32(tab_raw) & 511u)) & 511u));
     const uint32_t tab_sbase = smem_u32(s_tab);
 
-    // ---- phase 0: the routed ids are loaded first; one thread initialises the
-    // mbarriers and then issues the Phi rows and x (they need nothing) ----
-    const int my_id = (warp == 1 && lane < P.U) ? P.ids[lane % P.K] : 0;
+    // ---- launch: one thread initialises the mbarriers and issues the weight copies
+    // (expert directories, Phi rows); they are constant, so they go out before the
+    // wait for the previous kernel in the stream (programmatic dependent launch) ----
+    const bool plan_lane = warp == 1 && lane < P.U;
     if (tid == 0) {
-        for (int i = 0; i < kPhiBars + 4; i++) mbar_init(&s_bar[i], 1);
+        for (int i = 0; i < kNumBars; i++)
+            mbar_init(&s_bar[i], i == kZeroBar ? (uint32_t)n_zero_warps : i == kZBar ? (uint32_t)nzw : 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
         s_zto = 0;
     }
     __syncthreads();  // the mbarriers are initialised
-    // Roles: warp 1 plans this CTA's share and hands it to the last kStageWarps
-    // warps, which issue the staging copies; the other warps compute z rows as
-    // the Phi chunks land.  The three run side by side.
-    const int nrw = nwarps - kStageWarps;  // warps before the staging warps
-    const bool row_warp = warp < nrw;
     if (tid == 0) {
-        // both expert directories first: the routed units need them before anything else
+        // both expert directories first: the plan needs them before anything else
         const uint32_t dir_bytes = (uint32_t)P.E * kDirEntryBytes;
         const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
-        mbar_expect_tx(&s_bar[kPhiBars], 2 * dir_bytes);
+        mbar_expect_tx(&s_bar[kDirBar], 2 * dir_bytes);
         for (int p = 0; p < 2; p++)
-            bulk_g2s(s_dir + (size_t)p * dir_bytes, P.proj[p].blob + kHeaderBytes, dir_bytes, &s_bar[kPhiBars], keep);
+            bulk_g2s(s_dir + (size_t)p * dir_bytes, P.proj[p].blob + kHeaderBytes, dir_bytes, &s_bar[kDirBar], keep);
         for (int bi = 0; bi < kPhiBars; bi++) {
             const int ra = row0 + (nrows * bi) / kPhiBars, rbnd = row0 + (nrows * (bi + 1)) / kPhiBars;
-            const uint32_t bytes = (uint32_t)(rbnd - ra) * row_bytes + (bi == 0 ? row_bytes : 0);
+            const uint32_t bytes = (uint32_t)(rbnd - ra) * row_bytes;
             mbar_expect_tx(&s_bar[bi], bytes);
-            if (bi == 0) bulk_g2s(s_x, P.x, row_bytes, &s_bar[0], stream);
             for (int rr = ra; rr < rbnd;) {  // rows are contiguous inside a projection
                 const int p = rr / P.r, k = rr - p * P.r;
                 const int n = min(rbnd - rr, P.r - k);
@@ -388,6 +437,15 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                 rr += n;
             }
         }
+    }
+    // Everything below may read what the previous kernel in the stream wrote (x, the
+    // routing, the workspace's counter, tags and z rows, the outputs): wait for it.
+    // The next kernel may be launched now; its CTAs start as this kernel's CTAs exit.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int my_id = plan_lane ? P.ids[lane % P.K] : 0;
+    const float my_gw = plan_lane ? P.gw[lane % P.K] : 0.0f;
+    if (tid == 0) {
         // This launch's tag.  Every launch adds exactly G to the counter (one per
         // CTA, whatever happens later), so before this CTA's addition it holds G
         // times the number of earlier launches n plus fewer than G of this one's.
@@ -395,173 +453,20 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         // never that of the launch before.
         const unsigned long long before = atomicAdd(P.launches, 1ull);
         s_tag = (uint32_t)((before / (unsigned long long)P.G) % 0xFFFFFFFFull) + 1u;
-        mbar_arrive(&s_bar[kTagBar]);  // publishes s_tag to the row warps
-    }
-
-    // ---- routed units and this CTA's share (warp 1; one lane per unit, then per item).
-    // The other warps wait: this is short, and alone on the SM it is not slowed by them ----
-    if (warp == 1) {
-        const bool dir_ok = mbar_wait(&s_bar[kPhiBars], 0);
-        if (lane < P.U) unit_info(P, lane, dir_ok ? my_id : -1, s_dir, s_unit[lane]);
-        if (!dir_ok && lane == 0) s_abort = 1;
-        __syncwarp();
-        const bool is_unit = lane < P.U;
-        const int my_items = is_unit ? s_unit[lane].items : 0;
-        int incl = my_items;  // inclusive scan of items over units
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const int excl = incl - my_items;
-        const int Q = __shfl_sync(0xffffffffu, incl, 31);
-        const int q0 = share_begin(cta, Q, P.G);
-        int ni = share_begin(cta + 1, Q, P.G) - q0;
-        if (ni > P.items_max || ni > kMaxItems) {  // the blob's counts disagree with the plan's
-            if (lane == 0 && P.status) atomicOr(P.status, BITSMOE_ST_PLANMISMATCH);
-            ni = 0;
-        }
-        const bool bad = __any_sync(0xffffffffu, is_unit && s_unit[lane].e < 0);
-        // unit of item `lane`: the number of units that end at or before it
-        int my_u = 0;
-#pragma unroll
-        for (int v = 0; v < 32; v++) my_u += (v < P.U && __shfl_sync(0xffffffffu, incl, v) <= q0 + lane) ? 1 : 0;
-        my_u = min(my_u, P.U - 1);
-        const int S_u = __shfl_sync(0xffffffffu, excl, my_u & 31);
-        const bool valid = lane < ni;
-        Item it{};
-        int key = -1 - lane, g = 0, jb = -1, w = 0;  // member-word key of a plane word; unique otherwise
-        if (valid) {
-            const UnitInfo& U = s_unit[my_u];
-            const int l = q0 + lane - S_u;
-            const uint8_t* blob = P.proj[U.p].blob;
-            it.u = (int16_t)my_u;
-            if (l < U.pw) {
-                decode_pw(U, l, g, jb, w);
-                const uint32_t W = U.np[g] / 32;
-                it.ptr = blob + U.gbase[g] + 8ull * U.np[g] + 4ull * P.d_pad * ((uint64_t)jb * W + (uint64_t)w);
-                it.nf = 0;
-                key = (my_u << 24) | (g << 16) | w;
-            } else {
-                const int f = l - U.pw;
-                it.ptr = blob + U.gbase[0] + 6ull * U.np[0] + 2ull * kF16Item * (uint64_t)f * (uint64_t)P.d_pad;
-                it.nf = (int16_t)min(kF16Item, U.n16 - kF16Item * f);
-                it.w = (int16_t)f;
-            }
-        }
-        const bool plane = valid && it.nf == 0, oct = valid && it.nf > 0;
-        // runs of plane words: consecutive items whose words follow each other in the blob
-        const uint64_t my_ptr = (uint64_t)it.ptr;
-        const uint64_t prev_ptr = __shfl_up_sync(0xffffffffu, my_ptr, 1);
-        const int prev_plane = __shfl_up_sync(0xffffffffu, (int)plane, 1);
-        const bool cont = plane && lane > 0 && prev_plane && my_ptr == prev_ptr + 4ull * P.d_pad;
-        const unsigned bcont = __ballot_sync(0xffffffffu, cont), bplane = __ballot_sync(0xffffffffu, plane);
-        const unsigned brun = bplane & ~bcont;
-        if ((brun >> lane) & 1u) {
-            const unsigned stop = ~bcont & (lane == 31 ? 0u : ~((2u << lane) - 1u));  // first later item not continuing
-            Run R;
-            R.ptr = it.ptr;
-            R.a = lane;
-            R.len = (stop ? __ffs(stop) - 1 : 32) - lane;
-            s_run[__popc(brun & ((1u << lane) - 1u))] = R;
-        }
-        if (lane == 0) {
-            s_nrun = __popc(brun);
-            s_stage_bytes = 4u * (uint32_t)P.d_pad * (uint32_t)__popc(bplane);
-        }
-        named_barrier<2>(32 * (1 + kStageWarps));  // the plane runs are known: the staging warps copy them now
-        // first item of the same member word, and whether any of them is plane 0
-        int ref = lane, zp = 0;
-        const int z0 = plane && jb == 0;
-#pragma unroll
-        for (int k = 0; k < 32; k++) {
-            const int kk = __shfl_sync(0xffffffffu, key, k), kz = __shfl_sync(0xffffffffu, z0, k);
-            if (k < ni && kk == key) {
-                if (k < ref) ref = k;
-                zp |= kz;
-            }
-        }
-        const unsigned lt = (1u << lane) - 1u;
-        const bool newmw = plane && ref == lane;
-        const unsigned bm = __ballot_sync(0xffffffffu, newmw), bf = __ballot_sync(0xffffffffu, oct);
-        const int slot_new = __popc(bm & lt);
-        const int slot_ref = __shfl_sync(0xffffffffu, slot_new, ref);
-        const int slot = oct ? __popc(bf & lt) : slot_ref;
-        const int u_prev = __shfl_up_sync(0xffffffffu, my_u, 1);
-        const bool newseg = valid && (lane == 0 || u_prev != my_u);
-        const unsigned bs = __ballot_sync(0xffffffffu, newseg);
-        const int seg = __popc(bs & (lt | (1u << lane))) - 1;
-        if (valid) {
-            it.slot = (int16_t)slot;
-            s_item[lane] = it;
-            s_desc[lane] = plane ? make_uint2(tab_sbase + 512u * (uint32_t)slot, __float_as_uint((float)(1u << jb)))
-                                 : make_uint2(0u, 0u);
-        }
-        if (newmw) {
-            const UnitInfo& U = s_unit[my_u];
-            MemberWord M;
-            M.p = (int16_t)U.p;
-            M.g = (int16_t)g;
-            M.w = (int16_t)w;
-            M.nvalid = (int16_t)max(0, min(32, (int)U.n[g] - 32 * w));
-            M.zp = (int16_t)zp;
-            M.seg = (int16_t)seg;
-            s_mw[slot_new] = M;
-        }
-        {   // runs of member words in slot order: consecutive slots, same group, consecutive words
-            const unsigned below = bm & lt;
-            const int prev = below ? 31 - __clz(below) : 0;  // the previous slot's lane
-            const int pkey = __shfl_sync(0xffffffffu, key, prev);
-            const bool mcont = newmw && below != 0u && pkey == key - 1;
-            const unsigned bmc = __ballot_sync(0xffffffffu, mcont);
-            const unsigned bmr = bm & ~bmc;  // run starts
-            if ((bmr >> lane) & 1u) {
-                const unsigned after = lane == 31 ? 0u : ~((2u << lane) - 1u);
-                const unsigned nxt = bmr & after;
-                const unsigned span = nxt ? (after & ((1u << (__ffs(nxt) - 1)) - 1u)) : after;
-                const UnitInfo& U = s_unit[my_u];
-                MetaRun R;
-                R.meta = P.proj[U.p].blob + U.gbase[g];
-                R.np = U.np[g];
-                R.w = w;
-                R.slot = slot_new;
-                R.len = 1 + __popc(bm & span);
-                s_mrun[__popc(bmr & lt)] = R;
-            }
-            if (lane == 0) s_nmrun = __popc(bmr);
-        }
-        if (newseg) {
-            const unsigned above = bs & ~(lt | (1u << lane));
-            const int i1 = above ? __ffs(above) - 1 : ni;
-            const unsigned in_seg = (i1 >= 32 ? 0xffffffffu : ((1u << i1) - 1u)) & ~lt;
-            const unsigned octs = bf & in_seg;
-            Seg S;
-            S.u = my_u;
-            S.i0 = lane;
-            S.i1 = i1;
-            S.ip = octs ? __ffs(octs) - 1 : i1;
-            s_seg[seg] = S;
-        }
-        if (lane == 0) {
-            s_ni = ni;
-            s_nmw = __popc(bm);
-            s_nseg = __popc(bs);
-            s_meta_bytes = 256u * __popc(bm) + 48u * __popc(bf);
-            s_bad = bad;
-        }
-        named_barrier<3>(32 * (1 + kStageWarps));  // the rest of the plan: member words and octets
+        mbar_arrive(&s_bar[kTagBar]);  // publishes s_tag to the other warps
     }
 
     // ---- the outputs are sums of red.add contributions: the first n_zero CTAs zero
     // them and then publish this launch's tag; every CTA acquires those tags before
     // its first addition ----
-    const int rw = warp == 0 ? 0 : warp - 1, nrw1 = nrw - 1;  // index and count of the z-row warps
-    if (cta < P.n_zero && row_warp && warp != 1) {
+    if (cta < P.n_zero && zero_warp) {
+        if (!mbar_wait(&s_bar[kTagBar], 0)) s_abort = 1;  // s_tag
+        const int zw = warp == 0 ? 0 : warp - 1 - nzw;  // 0 .. n_zero_warps - 1
         const int nys = 2 * P.d_out;
         const int nye0 = P.proj[0].Ye ? P.K * P.d_out : 0, nye1 = P.proj[1].Ye ? P.K * P.d_out : 0;
         const int tot = nys + nye0 + nye1;
         const int a = share_begin(cta, tot, P.n_zero), b = share_begin(cta + 1, tot, P.n_zero);
-        for (int i = a + rw * 32 + lane; i < b; i += nrw1 * 32) {
+        for (int i = a + zw * 32 + lane; i < b; i += n_zero_warps * 32) {
             float* dst;
             if (i < P.d_out)
                 dst = P.proj[0].Ysum + i;
@@ -573,102 +478,337 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                 dst = P.proj[1].Ye + (i - nys - nye0);
             *dst = 0.0f;
         }
-        // the row warps' zeros are ordered before the tag by this CTA barrier and
-        // the cumulative release of the store (thread 0 wrote s_tag itself)
-        named_barrier<4>(nrw1 * 32);
-        if (tid == 0) st_release_u64(P.zero_tags + cta, (unsigned long long)s_tag);
+        // every zeroing warp's stores are ordered before the tag by its release
+        // arrival, thread 0's acquiring wait and the cumulative release store
+        // (thread 0 wrote s_tag itself)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_bar[kZeroBar]);
+        if (tid == 0) {
+            if (mbar_wait(&s_bar[kZeroBar], 0))
+                st_release_u64(P.zero_tags + cta, (unsigned long long)s_tag);
+            else
+                s_abort = 1;
+        }
+        __syncwarp();
     }
 
-    // ---- staging by the staging warp (bulk copies on one mbarrier): each run of plane
-    // words in one copy into [item slot][d_pad]; each run of member words' idx, scale
-    // and amp in one copy per array; each octet's idx and amp ----
-    if (!row_warp) {
-        named_barrier<2>(32 * (1 + kStageWarps));
-        // A CTA's bulk copies land in about the order they are issued, so copies
-        // issued now would land after this CTA's Phi rows anyway; issued now they
-        // would also take HBM time from other CTAs' Phi rows, which every CTA
-        // waits for.  So they are issued once this CTA's last Phi chunk has landed.
-        const bool phi_ok = mbar_wait(&s_bar[kPhiBars - 1], 0);
-        if (!phi_ok) s_abort = 1;
-        const int st = threadIdx.x - nrw * 32, nst = kStageWarps * 32;
-        const uint64_t stream = policy_evict_first();
-        uint64_t* bar = &s_bar[kPhiBars + 1];
-        if (st == 0) mbar_expect_tx(bar, s_stage_bytes);
-        __syncwarp();
-        for (int r = st; r < s_nrun; r += nst) {
-            const Run R = s_run[r];
-            bulk_g2s(s_planes + (size_t)R.a * P.d_pad, R.ptr, 4u * (uint32_t)P.d_pad * (uint32_t)R.len, bar, stream);
+    // ---- the plan of this CTA's share (warp 1): lane u handles routed unit u in its
+    // registers, cuts its part of the share into pieces and issues their plane
+    // copies itself ----
+    if (warp == 1) {
+        const bool dir_ok = mbar_wait(&s_bar[kDirBar], 0);
+        if (!dir_ok && lane == 0) s_abort = 1;
+        const bool is_unit = lane < P.U;
+        const int up = is_unit ? lane / P.K : 0, uj = is_unit ? lane - up * P.K : 0;
+        const bool valid_e = is_unit && dir_ok && my_id >= 0 && my_id < P.E;
+        UnitRegs R;
+        unit_regs(valid_e ? s_dir + ((size_t)up * P.E + my_id) * kDirEntryBytes : nullptr, R);
+        if (is_unit) s_unit[lane] = UnitRef{up, uj, my_gw};
+        const bool bad = __any_sync(0xffffffffu, is_unit && !(my_id >= 0 && my_id < P.E));
+        const int items = R.items;  // 0 for a lane past the units or an id out of range
+        int incl = items;           // inclusive scan of items over units
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        named_barrier<3>(32 * (1 + kStageWarps));
-        const int ni = s_ni;
-        bar = &s_bar[kPhiBars + 2];
-        if (st == 0) mbar_expect_tx(bar, s_meta_bytes);
-        __syncwarp();
-        for (int r = st; r < s_nmrun; r += nst) {
-            const MetaRun R = s_mrun[r];
-            const uint32_t n = (uint32_t)R.len;
-            bulk_g2s(s_midx + 32 * R.slot, R.meta + 64ull * R.w, 64u * n, bar, stream);                // idx
-            bulk_g2s(s_mscl + 32 * R.slot, R.meta + 2ull * R.np + 64ull * R.w, 64u * n, bar, stream);  // scale
-            bulk_g2s(s_mamp + 32 * R.slot, R.meta + 4ull * R.np + 128ull * R.w, 128u * n, bar, stream);  // amp
+        const int S = incl - items;  // this unit's first item in the concatenation
+        const int Q = __shfl_sync(0xffffffffu, incl, 31);
+        const int q0 = share_begin(cta, Q, P.G);
+        int ni = share_begin(cta + 1, Q, P.G) - q0;
+        if (ni > P.items_max || ni > kMaxItems) {  // the blob's counts disagree with the plan's
+            if (lane == 0 && P.status) atomicOr(P.status, BITSMOE_ST_PLANMISMATCH);
+            ni = 0;
         }
-        for (int i = st; i < ni; i += nst) {
-            const Item& it = s_item[i];
-            if (!it.nf) continue;
-            const UnitInfo& U = s_unit[it.u];
-            const uint8_t* gb = P.proj[U.p].blob + U.gbase[0];
-            uint8_t* dst = s_f16d + 48 * it.slot;
-            bulk_g2s(dst, gb + 16ull * it.w, 16u, bar, stream);
-            bulk_g2s(dst + 16, gb + 2ull * U.np[0] + 32ull * it.w, 32u, bar, stream);
-        }
-    }
-
-    // ---- phase 1: z rows of this CTA (row warps), each published with this launch's tag ----
-    if (row_warp && warp != 1) {
-        bool ok = nrows == 0 || (mbar_wait(&s_bar[kTagBar], 0) && mbar_wait(&s_bar[0], 0));  // 0 carries x
-        const unsigned long long tag_hi = (unsigned long long)s_tag << 32;
-        for (int rl = rw; ok && rl < nrows; rl += nrw1) {
-            int bi = 0;
-            while (bi + 1 < kPhiBars && rl >= (nrows * (bi + 1)) / kPhiBars) bi++;
-            if (!mbar_wait(&s_bar[bi], 0)) {
-                ok = false;
-                break;
+        const int q1 = q0 + ni;
+        // this unit's items inside the share: local indices [a, b)
+        const int a = max(q0, S) - S, b = min(q1, S + items) - S;
+        const bool live = a < b;
+        // pass 1: pieces, member words and staged bytes of this unit
+        int npc = 0, ntw = 0;
+        uint32_t plane_bytes = 0;
+#pragma unroll
+        for (int g = 1; g < kNumGroups; g++) {
+            const int W = (int)(R.np[g] >> 5), lo = (int)R.pw0[g], hi = lo + group_width(g) * W;
+            const int pa = max(a, lo), pb = min(b, hi);
+            if (pa < pb) {  // an empty group has lo == hi
+                const int nw = min(W, pb - pa);
+                npc++;
+                ntw += nw;
+                plane_bytes += 4u * (uint32_t)P.d_pad * (uint32_t)(pb - pa);
             }
-            const uint4* rowv = reinterpret_cast<const uint4*>(s_phi + (size_t)rl * row_bytes);
-            const uint4* xv = reinterpret_cast<const uint4*>(s_x);
-            float acc = 0.0f, acc1 = 0.0f;
-            for (int i8 = lane; i8 < P.d_in / 8; i8 += 32) dot8_f16(rowv[i8], xv[i8], acc, acc1);
-            acc = warp_sum(acc + acc1);
-            if (lane == 0) {
-                const int rr = row0 + rl, p = rr / P.r, k = rr - p * P.r;
-                st_relaxed_u64(P.zbuf + rr, tag_hi | __float_as_uint(acc));
-                if (P.proj[p].Z) P.proj[p].Z[k] = acc;
+        }
+        const int pa16 = max(a, R.pw);
+        const bool has16 = pa16 < b;  // fp16 octets [pw, items) meet the share
+        if (has16) npc++;
+        // one lane arms the plane barrier with the CTA's total before any copy is issued
+        uint32_t all_plane_bytes = plane_bytes;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) all_plane_bytes += __shfl_xor_sync(0xffffffffu, all_plane_bytes, o);
+        if (lane == 0) mbar_expect_tx(&s_bar[kPlaneBar], all_plane_bytes);
+        __syncwarp();
+        const uint64_t stream = policy_evict_first();
+        const uint8_t* blob = P.proj[up].blob;
+        // stage the plane words first (one bulk copy per piece): they are on the critical path
+#pragma unroll
+        for (int g = 1; g < kNumGroups; g++) {
+            const int W = (int)(R.np[g] >> 5), lo = (int)R.pw0[g], hi = lo + group_width(g) * W;
+            const int pa = max(a, lo), pb = min(b, hi);
+            if (pa < pb)
+                bulk_g2s(s_planes + (size_t)(S + pa - q0) * P.d_pad,
+                         blob + R.gbase[g] + 8ull * R.np[g] + 4ull * P.d_pad * (uint64_t)(pa - lo),
+                         4u * (uint32_t)P.d_pad * (uint32_t)(pb - pa), &s_bar[kPlaneBar], stream);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_bar[kCopyBar]);  // the z warps may start
+        int pinc = npc, tinc = ntw;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, pinc, o), w = __shfl_up_sync(0xffffffffu, tinc, o);
+            if (lane >= o) {
+                pinc += v;
+                tinc += w;
+            }
+        }
+        const int npieces = __shfl_sync(0xffffffffu, pinc, 31), ntab = __shfl_sync(0xffffffffu, tinc, 31);
+        const unsigned lt = (1u << lane) - 1u;
+        const unsigned blive = __ballot_sync(0xffffffffu, live);
+        // pass 2a: write the pieces
+        {
+            int k = pinc - npc, t = tinc - ntw;
+#pragma unroll
+            for (int g = 1; g < kNumGroups; g++) {
+                const int W = (int)(R.np[g] >> 5), lo = (int)R.pw0[g], hi = lo + group_width(g) * W;
+                const int pa = max(a, lo), pb = min(b, hi);
+                if (pa < pb) {
+                    const int nw = min(W, pb - pa);
+                    const int l0 = pa - lo;
+                    int wstart = 0;
+                    if (nw < W) {
+                        wstart = l0;
+                        while (wstart >= W) wstart -= W;  // l0 mod W (l0 < 8 W)
+                    }
+                    Piece X;
+                    X.gptr = blob + R.gbase[g];
+                    X.np = R.np[g];
+                    X.n = R.n[g];
+                    X.u = (int16_t)lane;
+                    X.g = (int16_t)g;
+                    X.l0 = (int16_t)l0;
+                    X.l1 = (int16_t)(pb - lo);
+                    X.slot0 = (int16_t)(S + pa - q0);
+                    X.tslot0 = (int16_t)t;
+                    X.nw = (int16_t)nw;
+                    X.wstart = (int16_t)wstart;
+                    X.W = (int16_t)W;
+                    X.pad_ = 0;
+                    s_piece[k++] = X;
+                    t += nw;
+                }
+            }
+            if (has16) {
+                Piece X;
+                X.gptr = blob + R.gbase[0];
+                X.np = R.np[0];
+                X.n = R.n[0];
+                X.u = (int16_t)lane;
+                X.g = 0;
+                X.l0 = (int16_t)(pa16 - R.pw);
+                X.l1 = (int16_t)(b - R.pw);
+                X.slot0 = (int16_t)(S + pa16 - q0);
+                X.tslot0 = (int16_t)t;
+                X.nw = X.wstart = X.W = X.pad_ = 0;
+                s_piece[k] = X;
+            }
+        }
+        if (live) {
+            Seg G;
+            G.u = lane;
+            G.i0 = S + a - q0;
+            G.ip = S + max(a, min(b, R.pw)) - q0;
+            G.i1 = S + b - q0;
+            G.t0 = tinc - ntw;
+            G.t1 = tinc;
+            s_seg[__popc(blive & lt)] = G;
+        }
+        __syncwarp();  // every lane has written its pieces
+        if (lane == 0) {
+            s_ni = ni;
+            s_nmw = ntab;
+            s_nseg = __popc(blive);
+            s_bad = bad;
+        }
+        // item descriptors: lane i finds the piece of item slot i
+        if (lane < ni) {
+            int k = 0;
+            while (k + 1 < npieces && s_piece[k + 1].slot0 <= lane) k++;
+            const Piece X = s_piece[k];
+            const int l = X.l0 + (lane - X.slot0);
+            Octet O;
+            O.gptr = X.gptr;
+            O.np = X.np;
+            O.l = 0;
+            O.nf = 0;
+            O.u = X.u;
+            O.pad_ = 0;
+            if (X.g > 0) {
+                int jb = 0, w = l;
+                while (w >= X.W) {  // l = jb * W + w, jb < 8
+                    w -= X.W;
+                    jb++;
+                }
+                int t = w - X.wstart;
+                if (t < 0) t += X.W;
+                s_desc[lane] = make_uint2(tab_sbase + 512u * (uint32_t)(X.tslot0 + t), __float_as_uint((float)(1u << jb)));
+            } else {
+                O.l = (int16_t)l;
+                O.nf = (int16_t)min(kF16Item, (int)X.n - kF16Item * l);
+                s_desc[lane] = make_uint2(0u, 0u);
+            }
+            s_oct[lane] = O;
+        }
+        // member words: lane t finds the bit-plane piece of table slot t
+        for (int t = lane; t < ntab; t += 32) {
+            int k = 0;
+            while (k + 1 < npieces && s_piece[k + 1].tslot0 <= t) k++;
+            const Piece X = s_piece[k];
+            int w = X.wstart + (t - X.tslot0);
+            if (w >= X.W) w -= X.W;
+            MemberWord M;
+            M.gptr = X.gptr;
+            M.np = X.np;
+            M.p = (int16_t)(X.u / P.K);
+            M.g = X.g;
+            M.w = (int16_t)w;
+            M.nvalid = (int16_t)max(0, min(32, (int)X.n - 32 * w));
+            M.zp = (int16_t)(w >= X.l0 && w < X.l1);  // plane 0 of word w is item w of the group
+            M.pad_ = 0;
+            s_mw[t] = M;
+        }
+        __syncwarp();  // the plan's shared-memory writes of every lane precede lane 0's release
+        if (lane == 0) mbar_arrive(&s_bar[kPlanBar]);
+        // the zeroing CTAs' tags (bounded waits), while the other warps compute z
+        const bool tag_ok = mbar_wait(&s_bar[kTagBar], 0);
+        if (lane < P.n_zero && (!tag_ok || !tag_wait(P.zero_tags + lane, (unsigned long long)s_tag))) s_abort = 1;
+        __syncwarp();
+    } else if (!z_warp) {
+        // the plan (bounded wait with back-off: these warps have nothing else to do,
+        // and polling would take issue slots from the planning and z warps)
+        if (!mbar_wait_sleep(&s_bar[kPlanBar], 0)) s_abort = 1;
+        // the metadata (idx, scale, amp) of every member word of the plan into shared
+        // memory, split over these warps (warp 0 and those after the z warps): one
+        // coalesced load per array and word
+        const int nmw_ = s_nmw, nlw = n_zero_warps, lw = warp == 0 ? 0 : warp - 1 - nzw;
+        for (int m = lw; m < nmw_; m += nlw) {
+            const MemberWord M = s_mw[m];
+            const int k = 32 * M.w + lane;  // member of the group (padding members carry zeros)
+            s_midx[32 * m + lane] = reinterpret_cast<const uint16_t*>(M.gptr)[k];
+            s_mscl[32 * m + lane] = reinterpret_cast<const uint16_t*>(M.gptr + 2ull * M.np)[k];
+            s_mamp[32 * m + lane] = reinterpret_cast<const float*>(M.gptr + 4ull * M.np)[k];
+        }
+    }
+
+
+
+    // ---- z rows of this CTA, split along d_in over the z warps: lane l of z warp zw
+    // owns 16-byte chunks l + 32 (zw + nzw m) of x (in registers) and accumulates
+    // every row's partial dot product over them; a multi-row warp reduction and a sum
+    // over the z warps give the rows, each published with this launch's tag ----
+    if (z_warp) {
+        const int zw = warp - 2;
+        // The z arithmetic (fp16 products, issue- and conversion-bound) starts once the
+        // planning warp has issued the plane copies, which everything after z waits for.
+        bool ok = mbar_wait_sleep(&s_bar[kCopyBar], 0);
+        ok = ok && (nrows == 0 || mbar_wait(&s_bar[kTagBar], 0));
+        const unsigned long long tag_hi = (unsigned long long)s_tag << 32;
+        const int nch = P.d_in / 8;
+        const uint4* xv = reinterpret_cast<const uint4*>(P.x);  // 16-byte chunks of x
+        const uint4 xc0 = lane + 32 * zw < nch ? xv[lane + 32 * zw] : make_uint4(0, 0, 0, 0);  // this lane's first
+        // chunk bi holds rows [nrows bi / 4, nrows (bi + 1) / 4): at most 8 of the at most
+        // kMaxRowsPerCta rows.  Per chunk: 8 row partials per lane, an 8-row warp reduction
+        // (lane l ends with row l & 7), and the warp's row sums into s_zpart.
+        for (int bi = 0; bi < kPhiBars; bi++) {
+            const int ra = (nrows * bi) / kPhiBars, rn = (nrows * (bi + 1)) / kPhiBars - ra;
+            if (!mbar_wait(&s_bar[bi], 0)) ok = false;
+            if (rn == 0) continue;
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) acc[i] = 0.0f;
+            for (int c = lane + 32 * zw; c < nch; c += 32 * nzw) {
+                const uint4 xc = c == lane + 32 * zw ? xc0 : xv[c];
+                const uint4* rp = reinterpret_cast<const uint4*>(s_phi + (size_t)ra * row_bytes) + c;
+                // rows in two groups of 4: the 4 loads first (rows past the chunk repeat its
+                // last row; their sums are never stored), then the FMAs interleaved over the
+                // 4 independent rows
+#pragma unroll
+                for (int g4 = 0; g4 < 8; g4 += 4) {
+                    uint4 v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) v[i] = rp[(size_t)min(g4 + i, rn - 1) * (row_bytes / 16)];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<0>(v[i].x, xc.x, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<1>(v[i].x, xc.x, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<0>(v[i].y, xc.y, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<1>(v[i].y, xc.y, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<0>(v[i].z, xc.z, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<1>(v[i].z, xc.z, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<0>(v[i].w, xc.w, acc[g4 + i]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) acc[g4 + i] = fma_f16x2<1>(v[i].w, xc.w, acc[g4 + i]);
+                }
+            }
+            const float part = warp_sum_rows8(acc, lane);
+            if (lane < rn) s_zpart[zw][ra + lane] = part;
+        }
+        if (nrows > 0) {  // at most kMaxRowsPerCta rows (the host checks it)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_bar[kZBar]);  // releases this warp's partial rows
+            if (zw == 0) {
+                if (!mbar_wait(&s_bar[kZBar], 0)) ok = false;
+                if (ok && lane < nrows) {
+                    float z = 0.0f;
+                    for (int w = 0; w < nzw; w++) z += s_zpart[w][lane];
+                    const int rr = row0 + lane, p = rr / P.r, k = rr - p * P.r;
+                    st_relaxed_u64(P.zbuf + rr, tag_hi | __float_as_uint(z));
+                    if (P.proj[p].Z) P.proj[p].Z[k] = z;
+                }
             }
         }
         if (!ok) s_abort = 1;
-        named_barrier<1>(nrw1 * 32);
-        if (tid == 0)
-            for (int bi = 0; bi < kPhiBars; bi++)  // every bulk copy into this CTA's shared memory has landed
-                if (!mbar_wait(&s_bar[bi], 0)) s_abort = 1;
     }
-    __syncthreads();
-    const int ni = s_ni, nmw = s_nmw, nseg = s_nseg;
-    const uint32_t tag = s_tag;
-
-    // ---- the outputs are zeroed, the planes and metadata have landed (bounded waits) ----
     if (tid == 0) {
-        for (int z = 0; z < P.n_zero; z++)
-            if (!tag_wait(P.zero_tags + z, (unsigned long long)tag)) s_abort = 1;
-        if (!mbar_wait(&s_bar[kPhiBars + 1], 0)) s_abort = 1;  // the staged planes
-        if (!mbar_wait(&s_bar[kPhiBars + 2], 0)) s_abort = 1;  // and metadata
+        // every bulk copy into this CTA's shared memory lands before it can exit
+        for (int bi = 0; bi < kPhiBars; bi++)
+            if (!mbar_wait(&s_bar[bi], 0)) s_abort = 1;
+        if (!mbar_wait(&s_bar[kPlaneBar], 0)) s_abort = 1;  // the staged planes
         if (s_bad && cta == 0 && P.status) atomicOr(P.status, BITSMOE_ST_BADEXPERT);
+        // This CTA's reads from HBM are done: while the experts are evaluated, pull
+        // its rows of the next layer's Phi into L2 for the next call.
+        if (!s_abort && P.next_phi[0] && P.next_phi[1])
+            for (int rr = row0; rr < row1;) {
+                const int p = rr / P.r, k = rr - p * P.r;
+                const int n = min(row1 - rr, P.r - k);
+                bulk_prefetch_l2(P.next_phi[p] + (size_t)k * P.d_in, (uint32_t)n * row_bytes);
+                rr += n;
+            }
     }
+    __syncwarp();
     __syncthreads();
     if (s_abort) {
         if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
         return;
     }
+    const int ni = s_ni, nseg = s_nseg;
+    const uint32_t tag = s_tag;
 
     // ---- c_k = a_k s_k z_k, the tables and the zero-point share: a warp per member word ----
+    const int nmw = s_nmw;
     for (int m = warp; m < nmw; m += nwarps) {
         const MemberWord M = s_mw[m];
         const int k = s_midx[32 * m + lane];
@@ -679,8 +819,8 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         // entry e of table tb = the sum of c over the set bits of e (members 4 tb .. 4 tb + 3)
         const int e = lane & 15;
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const int tb = (lane >> 4) + 2 * q;
+        for (int qq = 0; qq < 4; qq++) {
+            const int tb = (lane >> 4) + 2 * qq;
             const float c0 = __shfl_sync(0xffffffffu, c, 4 * tb), c1 = __shfl_sync(0xffffffffu, c, 4 * tb + 1);
             const float c2 = __shfl_sync(0xffffffffu, c, 4 * tb + 2), c3 = __shfl_sync(0xffffffffu, c, 4 * tb + 3);
             s_tab[128 * m + 16 * tb + e] =
@@ -692,41 +832,34 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
     }
     for (int ch = tid; ch < ni * kF16Item; ch += nthreads) {
         const int i = ch / kF16Item, m = ch - i * kF16Item;
-        const Item& it = s_item[i];
-        if (!it.nf) continue;
-        const uint8_t* fd = s_f16d + 48 * it.slot;
-        const int k = reinterpret_cast<const uint16_t*>(fd)[m];
+        const Octet O = s_oct[i];
+        if (!O.nf) continue;
         float c = 0.0f;
-        if (m < it.nf && k < P.r)
-            c = reinterpret_cast<const float*>(fd + 16)[m] * z_poll(P.zbuf + s_unit[it.u].p * P.r + k, tag, &s_zto);
-        s_c16[kF16Item * it.slot + m] = c;
+        if (m < O.nf) {
+            const int k = reinterpret_cast<const uint16_t*>(O.gptr)[kF16Item * O.l + m];
+            if (k < P.r)
+                c = reinterpret_cast<const float*>(O.gptr + 2ull * O.np)[kF16Item * O.l + m] *
+                    z_poll(P.zbuf + s_unit[O.u].p * P.r + k, tag, &s_zto);
+        }
+        s_c16[kF16Item * i + m] = c;
     }
+    __syncwarp();
     __syncthreads();
     if (s_zto) {
         if (tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
         return;
     }
-    // This CTA has every z row it needs, so the Phi reads of this launch are all
-    // but done: HBM is free while the experts are evaluated, so pull this CTA's
-    // rows of the next layer's Phi into L2 for the next call.
-    if (tid == 0 && P.next_phi[0] && P.next_phi[1])
-        for (int rr = row0; rr < row1;) {
-            const int p = rr / P.r, k = rr - p * P.r;
-            const int n = min(row1 - rr, P.r - k);
-            bulk_prefetch_l2(P.next_phi[p] + (size_t)k * P.d_in, (uint32_t)n * row_bytes);
-            rr += n;
-        }
 
     // ---- lookups: warps own 32-row tiles; a segment's rows go to Y_e and, times g, to Y_sum ----
     for (int s = 0; s < nseg; s++) {
         const Seg S = s_seg[s];
-        const UnitInfo& U = s_unit[S.u];
+        const UnitRef U = s_unit[S.u];
         const int p = U.p;
         float* ye = P.proj[p].Ye ? P.proj[p].Ye + (size_t)U.j * P.d_out : nullptr;
         float* ys = P.proj[p].Ysum;
         const float gj = U.g;
-        // this CTA's zero-point share of the unit (member words in slot order)
-        const float zps = warp_sum(lane < nmw && s_mw[lane].seg == s ? s_zpmw[lane] : 0.0f);
+        // this CTA's zero-point share of the unit (its member words are slots [t0, t1), at most 32)
+        const float zps = warp_sum(S.t0 + lane < S.t1 ? s_zpmw[S.t0 + lane] : 0.0f);
         for (int t = warp; t < P.n_rb; t += nwarps) {
             const uint32_t* pl = s_planes + t * kRB + lane;  // [item slot][d_pad]
             float acc = 0.0f;
@@ -751,11 +884,12 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             }
             const int row = t * kRB + lane;
             for (int i = S.ip; i < S.i1; i++) {  // fp16 octets, rows read in place
-                const Item& it = s_item[i];
-                const uint16_t* w16 = reinterpret_cast<const uint16_t*>(it.ptr);
-                for (int m = 0; m < it.nf; m++)
-                    acc = fmaf(s_c16[kF16Item * it.slot + m],
-                               __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row])), acc);
+                const Octet O = s_oct[i];
+                const uint16_t* w16 = reinterpret_cast<const uint16_t*>(O.gptr + 6ull * O.np) +
+                                      (size_t)kF16Item * O.l * P.d_pad;
+                for (int m = 0; m < O.nf; m++)
+                    acc = fmaf(s_c16[kF16Item * i + m], __half2float(__ushort_as_half(w16[(size_t)m * P.d_pad + row])),
+                               acc);
             }
             if (row < P.d_out) {
                 const float y = acc - zps;
@@ -858,15 +992,16 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     if ((uint64_t)P.G * (uint64_t)std::max<long long>(q_max, 2ll * std::max(P.r, P.d_out) * (P.K + 1)) >= (1ull << 32))
         return L;  // the 32-bit share arithmetic
     if (2ull * kDirEntryBytes * P.E >= (1u << 20)) return L;  // one mbarrier transaction count
+    // the staged planes of one CTA are one mbarrier transaction count
+    if (4ull * P.d_pad * P.items_max >= (1u << 20)) return L;
     const int im = std::max(1, P.items_max);
     const int phi_rows = (2 * P.r + P.G - 1) / P.G;
-    P.sm_x = 0;
-    P.sm_dir = align_up(2ull * P.d_in, 128);
+    if (phi_rows > kMaxRowsPerCta) return L;  // one multi-row warp reduction of z per CTA
+    P.sm_dir = 0;
     P.sm_phi = align_up(P.sm_dir + 2ull * kDirEntryBytes * P.E, 128);
     P.sm_planes = align_up(P.sm_phi + (uint64_t)phi_rows * P.d_in * 2, 128);
-    P.sm_mw = align_up(P.sm_planes + 128ull * P.n_rb * im, 128);
-    P.sm_f16 = align_up(P.sm_mw + 256ull * im, 16);
-    P.sm_c16 = align_up(P.sm_f16 + 48ull * im, 16);
+    P.sm_meta = align_up(P.sm_planes + 128ull * P.n_rb * im, 16);
+    P.sm_c16 = align_up(P.sm_meta + 256ull * im, 16);
     P.sm_tab = align_up(P.sm_c16 + 32ull * im, 16);
     P.sm_end = align_up(P.sm_tab + 512ull + 512ull * im, 16);  // + 512: tables realigned in the kernel
     L.smem = P.sm_end;
@@ -924,8 +1059,12 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
     cfg.dynamicSmemBytes = L.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    // Programmatic dependent launch: consecutive calls in a stream overlap the next
+    // launch with this one's tail.  Every CTA must be resident at once (the z rows and
+    // zeroing tags are exchanged between CTAs): one CTA per SM, which the shared-memory
+    // size enforces, and every wait between CTAs is bounded (BITSMOE_ST_TIMEOUT).
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, k_layer_t1, P);
