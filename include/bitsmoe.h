@@ -80,6 +80,8 @@ extern "C" {
 #define BITSMOE_ST_BADEXPERT 4   /* a routed expert id outside [0, E): zero Y_e row, left out of Y_sum */
 #define BITSMOE_ST_TIMEOUT 8     /* a bounded device wait gave up; outputs of that call are invalid */
 #define BITSMOE_ST_PLANMISMATCH 16 /* device widths disagree with the plan's widths */
+#define BITSMOE_ST_BOUNDS 32       /* bounds-checked build only: a computed index fell outside its
+                                      buffer; that access was skipped (outputs of the call invalid) */
 
 typedef struct {
     int32_t d_in;      /* input width of the projection (rows of Phi) */

@@ -13,10 +13,13 @@ import os
 import numpy as np
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbitsmoe.so")
+# BITSMOE_CHECKED=1 selects the bounds-checked build (libbitsmoe_checked.so): every
+# computed index of the expert kernels is checked, a violation sets ST_BOUNDS.
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libbitsmoe_checked.so" if os.environ.get("BITSMOE_CHECKED") == "1" else "libbitsmoe.so")
 
 OK, EINVAL, EWIDTH, ESIZE, ECUDA, EFORMAT, ENOMEM = 0, -1, -2, -3, -4, -5, -6
-ST_NONFINITE, ST_BADSCALE, ST_BADEXPERT, ST_TIMEOUT, ST_PLANMISMATCH = 1, 2, 4, 8, 16
+ST_NONFINITE, ST_BADSCALE, ST_BADEXPERT, ST_TIMEOUT, ST_PLANMISMATCH, ST_BOUNDS = 1, 2, 4, 8, 16, 32
 
 # Every symbol include/bitsmoe.h declares.
 EXPORTS = (
@@ -52,7 +55,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(_LIB_PATH):
-            raise RuntimeError(f"{_LIB_PATH} is missing: build it with mixed_precision_decode_b200.build.build()")
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with mixed_precision_decode_b200.build.build()"
+                               f" (checked=True for the bounds-checked build)")
         L = ctypes.CDLL(_LIB_PATH)
         vp, u64, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int32
         sig = {

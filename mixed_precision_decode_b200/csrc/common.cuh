@@ -145,6 +145,20 @@ __device__ __forceinline__ uint32_t quantise(float p, int b, uint16_t sh, int& s
     return (uint32_t)f;
 }
 
+// Bounds checks of the checked build (compiled with -DBITSMOE_CHECKED): an
+// index i into a buffer of n elements (or a byte range ending at i) is checked
+// before use; outside, BITSMOE_ST_BOUNDS is OR-ed into the status word and the
+// caller skips the access.  In the normal build the check is the constant true.
+#ifdef BITSMOE_CHECKED
+__device__ __forceinline__ bool in_bounds(uint64_t i, uint64_t n, int32_t* status) {
+    if (i < n) return true;
+    if (status) atomicOr(status, BITSMOE_ST_BOUNDS);
+    return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(uint64_t, uint64_t, int32_t*) { return true; }
+#endif
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

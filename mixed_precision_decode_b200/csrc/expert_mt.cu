@@ -39,6 +39,10 @@ constexpr long long kMtWaitNs = 2000000000LL;
 
 struct MtParams {
     const uint8_t* blob;
+    uint64_t blob_bytes;
+    uint32_t stage_words;  // words of the staging buffer
+    uint32_t c_floats;     // floats of the c rows' buffer
+    int n_pairs;           // T * K: rows of Y_e
     RouteWS rw;
     float* Ye;
     int32_t* status;
@@ -275,6 +279,9 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
             const uint8_t* src = P.blob + s_ex.gbase[g] + 8ull * s_ex.np[g] +
                                  4ull * ((uint64_t)(q - qg) * (uint64_t)P.d_pad + 32ull * tile0) + 16ull * piece;
             const uint32_t dst = mt_smem_u32(s_stage + s_ex.stage_off[g] + (q - qg) * 32u * ntl + 4u * piece);
+            if (!in_bounds(s_ex.stage_off[g] + (q - qg) * 32u * ntl + 4u * piece + 3u, P.stage_words, P.status) ||
+                !in_bounds((uint64_t)(src - P.blob) + 15u, P.blob_bytes, P.status))
+                continue;
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -294,7 +301,8 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                 const int pr = u < nt ? P.rw.pairs[pq + u] : -1;
                 s_pair[u] = pr;
                 s_zp[u] = pr >= 0 ? P.rw.zp[pr] : 0.0f;
-                if (pr >= 0 && members > 0)
+                if (pr >= 0 && members > 0 && in_bounds((uint64_t)(u + 1) * members - 1, P.c_floats, P.status) &&
+                    in_bounds(pr, (uint64_t)P.n_pairs, P.status))
                     mt_bulk(s_c + (size_t)u * members, P.rw.cvals + (size_t)pr * P.rw.ldc, 4u * members, &s_cbar);
             }
             if (!mt_mbar_wait(&s_cbar, cphase)) s_fail = 1;
@@ -468,7 +476,8 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
             }
 #pragma unroll
             for (int u = 0; u < kMtTok; u++)
-                if (u < nt) P.Ye[(size_t)s_pair[u] * P.d_out + row] = y[u];
+                if (u < nt && in_bounds(s_pair[u], (uint64_t)P.n_pairs, P.status))
+                    P.Ye[(size_t)s_pair[u] * P.d_out + row] = y[u];
         }
     }
 }
@@ -498,6 +507,8 @@ int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, co
 
     MtParams P{};
     P.blob = (const uint8_t*)blob;
+    P.blob_bytes = p->blob_bytes;
+    P.n_pairs = npairs;
     P.rw = rw;
     P.Ye = Ye;
     P.status = status;
@@ -535,6 +546,8 @@ int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, co
     P.sm_stage = 0;
     P.sm_c = (uint32_t)roundup(4ull * tile_words * tpc, 128);
     P.sm_tab = P.sm_c + (uint32_t)roundup(4ull * kMtTok * p->max_members_padded, 128);
+    P.stage_words = (uint32_t)(tile_words * tpc);
+    P.c_floats = (uint32_t)(kMtTok * p->max_members_padded);
     const size_t smem = P.sm_tab + kMtWarps * 2048 + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_expert_mt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return set_cuda_error(e);

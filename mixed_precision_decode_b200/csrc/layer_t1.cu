@@ -61,6 +61,7 @@ static_assert(8 * (1 + kMaxZeroCtas) <= 256, "the workspace head is 256 bytes");
 
 struct T1Proj {
     const uint8_t* blob;
+    uint64_t blob_bytes;
     const uint16_t* phi_t;
     float* Z;     // [r] or null
     float* Ye;    // [K][d_out] or null
@@ -432,8 +433,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             for (int rr = ra; rr < rbnd;) {  // rows are contiguous inside a projection
                 const int p = rr / P.r, k = rr - p * P.r;
                 const int n = min(rbnd - rr, P.r - k);
-                bulk_g2s(s_phi + (size_t)(rr - row0) * row_bytes, P.proj[p].phi_t + (size_t)k * P.d_in,
-                         (uint32_t)n * row_bytes, &s_bar[bi], stream);
+                if (in_bounds((uint64_t)(rr - row0 + n) * row_bytes - 1, P.sm_planes - P.sm_phi, P.status) &&
+                    in_bounds((uint64_t)(k + n) * P.d_in - 1, (uint64_t)P.r * P.d_in, P.status))
+                    bulk_g2s(s_phi + (size_t)(rr - row0) * row_bytes, P.proj[p].phi_t + (size_t)k * P.d_in,
+                             (uint32_t)n * row_bytes, &s_bar[bi], stream);
                 rr += n;
             }
         }
@@ -554,7 +557,10 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         for (int g = 1; g < kNumGroups; g++) {
             const int W = (int)(R.np[g] >> 5), lo = (int)R.pw0[g], hi = lo + group_width(g) * W;
             const int pa = max(a, lo), pb = min(b, hi);
-            if (pa < pb)
+            if (pa < pb &&
+                in_bounds((uint64_t)(S + pb - q0) * P.d_pad * 4 - 1, 4ull * P.items_max * P.d_pad, P.status) &&
+                in_bounds(R.gbase[g] + 8ull * R.np[g] + 4ull * P.d_pad * (uint64_t)(pb - lo) - 1,
+                          P.proj[up].blob_bytes, P.status))
                 bulk_g2s(s_planes + (size_t)(S + pa - q0) * P.d_pad,
                          blob + R.gbase[g] + 8ull * R.np[g] + 4ull * P.d_pad * (uint64_t)(pa - lo),
                          4u * (uint32_t)P.d_pad * (uint32_t)(pb - pa), &s_bar[kPlaneBar], stream);
@@ -602,7 +608,9 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                     X.wstart = (int16_t)wstart;
                     X.W = (int16_t)W;
                     X.pad_ = 0;
-                    s_piece[k++] = X;
+                    if (in_bounds(k, kMaxItems, P.status) && in_bounds(t + nw - 1, (uint64_t)P.items_max, P.status))
+                        s_piece[k] = X;
+                    k++;
                     t += nw;
                 }
             }
@@ -618,7 +626,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                 X.slot0 = (int16_t)(S + pa16 - q0);
                 X.tslot0 = (int16_t)t;
                 X.nw = X.wstart = X.W = X.pad_ = 0;
-                s_piece[k] = X;
+                if (in_bounds(k, kMaxItems, P.status)) s_piece[k] = X;
             }
         }
         if (live) {
@@ -659,6 +667,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
                 }
                 int t = w - X.wstart;
                 if (t < 0) t += X.W;
+                if (!in_bounds(X.tslot0 + t, (uint64_t)P.items_max, P.status)) t = -X.tslot0;  // slot 0: a wrong sum, no stray access
                 s_desc[lane] = make_uint2(tab_sbase + 512u * (uint32_t)(X.tslot0 + t), __float_as_uint((float)(1u << jb)));
             } else {
                 O.l = (int16_t)l;
@@ -702,6 +711,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         for (int m = lw; m < nmw_; m += nlw) {
             const MemberWord M = s_mw[m];
             const int k = 32 * M.w + lane;  // member of the group (padding members carry zeros)
+            if (!in_bounds(m, (uint64_t)P.items_max, P.status) || !in_bounds(k, M.np, P.status)) continue;
             s_midx[32 * m + lane] = reinterpret_cast<const uint16_t*>(M.gptr)[k];
             s_mscl[32 * m + lane] = reinterpret_cast<const uint16_t*>(M.gptr + 2ull * M.np)[k];
             s_mamp[32 * m + lane] = reinterpret_cast<const float*>(M.gptr + 4ull * M.np)[k];
@@ -771,7 +781,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             if (lane == 0) mbar_arrive(&s_bar[kZBar]);  // releases this warp's partial rows
             if (zw == 0) {
                 if (!mbar_wait(&s_bar[kZBar], 0)) ok = false;
-                if (ok && lane < nrows) {
+                if (ok && lane < nrows && in_bounds(row0 + lane, 2ull * P.r, P.status)) {
                     float z = 0.0f;
                     for (int w = 0; w < nzw; w++) z += s_zpart[w][lane];
                     const int rr = row0 + lane, p = rr / P.r, k = rr - p * P.r;
@@ -813,7 +823,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
         const MemberWord M = s_mw[m];
         const int k = s_midx[32 * m + lane];
         float c = 0.0f;
-        if (lane < M.nvalid && k < P.r)
+        if (lane < M.nvalid && k < P.r && in_bounds(M.p * P.r + k, 2ull * P.r, P.status))
             c = s_mamp[32 * m + lane] * __half2float(__ushort_as_half(s_mscl[32 * m + lane])) *
                 z_poll(P.zbuf + M.p * P.r + k, tag, &s_zto);
         // entry e of table tb = the sum of c over the set bits of e (members 4 tb .. 4 tb + 3)
@@ -865,6 +875,7 @@ __global__ void __launch_bounds__(kT1MaxThreads, 1) k_layer_t1(const T1Params P)
             float acc = 0.0f;
 #pragma unroll 4
             for (int i = S.i0; i < S.ip; i++) {
+                if (!in_bounds((uint64_t)i * P.d_pad + t * kRB + lane, (uint64_t)P.items_max * P.d_pad, P.status)) break;
                 const uint2 d = s_desc[i];
                 const uint32_t word = pl[i * P.d_pad];
                 // entry offsets (nibble x 4 bytes): even nibbles in the bytes of lo, odd in hi;
@@ -911,9 +922,11 @@ struct T1Layout {
     int threads;
 };
 
-static int g_num_sms = 0;
-static int g_max_smem = 0;
-static int g_static_smem = -1;
+// Limits of the current device that the launch shape depends on, looked up once per
+// device (a process may drive GPUs of different SM counts).
+struct DeviceInfo {
+    int num_sms, max_smem, static_smem;
+};
 
 // Largest dynamic shared memory size k_layer_t1 has been granted on each
 // device, so that a launch asks the runtime again only when it needs more.
@@ -934,15 +947,26 @@ static cudaError_t grant_smem(int bytes) {
     return cudaSuccess;
 }
 
-static bool device_info() {
-    if (g_num_sms > 0 && g_static_smem >= 0) return true;
+static std::mutex g_devinfo_mu;
+static DeviceInfo g_devinfo[kMaxDevices];
+static bool g_devinfo_ok[kMaxDevices];
+
+static bool device_info(DeviceInfo* out) {
     int dev;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    if (cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-    if (cudaDeviceGetAttribute(&g_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, k_layer_t1) != cudaSuccess) return false;
-    g_static_smem = (int)fa.sharedSizeBytes;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lock(g_devinfo_mu);
+    if (!g_devinfo_ok[dev]) {
+        DeviceInfo d{};
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+        if (cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return false;
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, k_layer_t1) != cudaSuccess) return false;
+        d.static_smem = (int)fa.sharedSizeBytes;
+        g_devinfo[dev] = d;
+        g_devinfo_ok[dev] = true;
+    }
+    *out = g_devinfo[dev];
     return true;
 }
 
@@ -973,7 +997,8 @@ static uint32_t align_up(uint64_t v, uint64_t a) { return (uint32_t)roundup(v, a
 static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     T1Layout L{};
     L.ok = false;
-    if (!device_info()) return L;
+    DeviceInfo dv;
+    if (!device_info(&dv)) return L;
     T1Params& P = L.P;
     P.d_in = g->dims.d_in;
     P.d_out = g->dims.d_out;
@@ -984,7 +1009,7 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     P.U = 2 * P.K;
     if (u->dims.d_out != P.d_out || u->dims.rank != P.r || u->dims.d_in != P.d_in) return L;
     if (P.U > kMaxUnits || P.d_in % 8 || P.d_in > 8192 || P.d_pad % kRB) return L;
-    P.G = g_num_sms;
+    P.G = dv.num_sms;
     P.n_rb = P.d_pad / kRB;
     const long long q_max = (long long)P.K * (expert_items_max(g) + expert_items_max(u));
     P.items_max = (int)((q_max + P.G - 1) / P.G);
@@ -1005,7 +1030,7 @@ static T1Layout t1_layout(const bitsmoe_plan* g, const bitsmoe_plan* u) {
     P.sm_tab = align_up(P.sm_c16 + 32ull * im, 16);
     P.sm_end = align_up(P.sm_tab + 512ull + 512ull * im, 16);  // + 512: tables realigned in the kernel
     L.smem = P.sm_end;
-    if (L.smem + (size_t)g_static_smem > (size_t)g_max_smem) return L;
+    if (L.smem + (size_t)dv.static_smem > (size_t)dv.max_smem) return L;
     L.threads = 32 * choose_warps(P.n_rb);
     // workspace: the launch counter and the zeroing CTAs' tags (a 256-byte head),
     // then the tagged z rows.  All of it persists between calls (a stale z word
@@ -1031,6 +1056,7 @@ int layer_forward_fused_t1(const bitsmoe_proj_io** io, const uint16_t* X, const 
     T1Params P = L.P;
     for (int j = 0; j < 2; j++) {
         P.proj[j].blob = (const uint8_t*)io[j]->blob;
+        P.proj[j].blob_bytes = io[j]->plan->blob_bytes;
         P.proj[j].phi_t = io[j]->phi_t;
         P.proj[j].Z = io[j]->Z;
         P.proj[j].Ye = io[j]->Y_experts;

@@ -35,6 +35,18 @@ def test_exports_every_declared_symbol(B):
     assert B.version() == 100
 
 
+def test_checked_build_exports_the_same_symbols(B):
+    """The bounds-checked library is the same C ABI (only the kernels differ)."""
+    import ctypes
+    from mixed_precision_decode_b200 import build
+    path = build.build(checked=True)
+    L = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(L, name), name
+    L.bitsmoe_version.restype = ctypes.c_int
+    assert L.bitsmoe_version() == 100
+
+
 def _widths(rng, E, r):
     return rng.choice(np.array([0, 1, 2, 3, 4, 6, 8, 16], np.uint8), size=(E, r))
 
