@@ -6,12 +6,19 @@
 // One CTA computes a 128 (rows of Phi^T) x N (tokens, padded to 16) tile over
 // one K slice; the 8 CTAs of a cluster take the 8 K slices of the same tile and
 // add their fp32 partial tiles through distributed shared memory in rank order
-// (deterministic, no workspace).  Operands are copied with cp.async into the
-// canonical K-major no-swizzle layout (8-row x 16-byte core matrices), one
-// thread issues tcgen05.mma (kind::f16, fp32 accumulation in tensor memory),
-// tcgen05.commit signals an mbarrier, and four warps read the accumulator back
-// with tcgen05.ld.  The step is HBM-bound (64 flop per Phi byte at T = 64).
+// (deterministic, no workspace) by pushing rows into the owning rank's shared
+// memory with remote stores.  Operands arrive by 2-D TMA tiles
+// (cp.async.bulk.tensor, 64 K-elements x rows, 128-byte swizzle; tokens past T
+// read as zeros), one stage of K = 64 per mbarrier, all stages of a round issued
+// at once; one thread issues each stage's tcgen05.mma (kind::f16, fp32
+// accumulation in tensor memory) as soon as that stage has landed, so the loads
+// of later stages overlap the MMAs of earlier ones; tcgen05.commit signals an
+// mbarrier and four warps read the accumulator back with tcgen05.ld.  The step
+// is HBM-bound (64 flop per Phi byte at T = 64).
+#include <cuda.h>
+
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -22,6 +29,7 @@ constexpr int kTcM = 128;             // rows of Phi^T per tile
 constexpr int kTcK = 64;              // K per stage (4 MMAs of K = 16)
 constexpr int kTcCluster = 8;         // K slices per tile
 constexpr int kTcMaxStages = 4;       // stages resident at once
+constexpr int kTcBulkCols = 32;       // token tiles up to this width reduce by bulk copies (measured: faster at 16, slower at 64)
 constexpr long long kTcWaitNs = 2000000000LL;
 
 struct TcParams {
@@ -34,16 +42,19 @@ struct TcParams {
     int t_base;       // first token of the tile
     int k_per_cta;    // K slice length (multiple of kTcK)
     uint32_t stage_bytes;
+    uint32_t recv_off;  // byte offset of the receive slices (bulk reduction)
 };
 
 __device__ __forceinline__ uint32_t tc_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-// Shared-memory matrix descriptor: start, leading (K-adjacent core matrices)
-// and stride (M/N-adjacent 8-row groups) byte offsets, descriptor version 1,
-// no swizzle.
-__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzled
+// layout that a TMA tile of 64 fp16 K-elements per row writes: start address,
+// leading byte offset (unused for this layout; 16 B), stride byte offset between
+// 8-row groups (1024 B), descriptor version 1, layout type 2 (128-byte swizzle).
+// A K step of 16 elements inside the 128-byte row advances the start by 32 B.
+__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024u >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, both K-major.
@@ -51,8 +62,13 @@ __host__ __device__ constexpr uint32_t tc_idesc(int m, int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-__device__ __forceinline__ void tc_cp16(uint32_t dst, const void* src, uint32_t bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+// 2-D TMA tile load (no multicast) into shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tc_tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
 }
 
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
@@ -72,9 +88,12 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const TcParams P) {
+__global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const TcParams P, const __grid_constant__ CUtensorMap tmA,
+                                                           const __grid_constant__ CUtensorMap tmB) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ uint64_t s_mbar;
+    __shared__ uint64_t s_mbar;               // the MMAs of a round are done
+    __shared__ uint64_t s_lbar[kTcMaxStages];  // stage st of a round has landed
+    __shared__ uint64_t s_rbar;                // this rank's 8 row slices have arrived (bulk reduction)
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -96,49 +115,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const TcParams P) {
     }
     if (tid == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mbar));
+        for (int st = 0; st < kTcMaxStages; st++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem(&s_lbar[st])));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem(&s_rbar)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (P.n_pad <= kTcBulkCols)  // armed before any remote copy can arrive (the cluster barrier below)
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_smem(&s_rbar)),
+                         "r"((uint32_t)(kTcCluster * 16 * 4) * (uint32_t)P.n_pad)
+                         : "memory");
         s_fail = 0;
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    // This CTA's mbarriers are initialised: arrive now, wait only before the first
+    // remote access below (a CTA of the cluster may start later than this one).
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     const uint32_t tmem = s_tmem;
     const uint32_t idesc = tc_idesc(kTcM, n_pad);
 
-    uint32_t phase = 0;
+    const uint32_t a_bytes = kTcM * kTcK * 2, b_bytes = (uint32_t)n_pad * kTcK * 2;
+    uint32_t round = 0;
     bool accumulate = false;
-    for (int kc = kbeg; kc < kend && !s_fail; kc += kTcK * kTcMaxStages) {
+    for (int kc = kbeg; kc < kend; kc += kTcK * kTcMaxStages, round++) {
         const int nst = min(kTcMaxStages, (kend - kc) / kTcK);
-        // operands of nst stages into the K-major core-matrix layout (8 rows x 16 B per core matrix;
-        // core matrix (row group i, K group j) at (8 i + j) * 128 bytes)
-        for (int st = 0; st < nst; st++) {
-            const int k0 = kc + st * kTcK;
-            const uint32_t a_s = sbase + (uint32_t)st * P.stage_bytes, b_s = a_s + kTcM * kTcK * 2;
-            for (int c = tid; c < kTcM * 8; c += kTcThreads) {
-                const int rr = c >> 3, j = c & 7;
-                tc_cp16(a_s + (uint32_t)(((rr >> 3) * 8 + j) * 128 + (rr & 7) * 16),
-                        P.phi_t + (size_t)(m0 + rr) * P.d_in + k0 + 8 * j, 16u);
-            }
-            for (int c = tid; c < n_pad * 8; c += kTcThreads) {
-                const int tt = c >> 3, j = c & 7;
-                const int t = P.t_base + tt;
-                const bool ok = t < P.T;
-                tc_cp16(b_s + (uint32_t)(((tt >> 3) * 8 + j) * 128 + (tt & 7) * 16),
-                        ok ? (const void*)(P.X + (size_t)t * P.d_in + k0 + 8 * j) : (const void*)P.X, ok ? 16u : 0u);
-            }
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
-        __syncthreads();
         if (tid == 0) {
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            // every stage of the round at once: A = rows m0.. of Phi^T, B = the token tile
             for (int st = 0; st < nst; st++) {
-                const uint32_t a_s = sbase + (uint32_t)st * P.stage_bytes, b_s = a_s + kTcM * kTcK * 2;
+                const int k0 = kc + st * kTcK;
+                const uint32_t a_s = sbase + (uint32_t)st * P.stage_bytes, b_s = a_s + a_bytes;
+                const uint32_t lb = tc_smem(&s_lbar[st]);
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(lb), "r"(a_bytes + b_bytes)
+                             : "memory");
+                tc_tma2d(a_s, &tmA, k0, m0, lb);
+                tc_tma2d(b_s, &tmB, k0, P.t_base, lb);
+            }
+            // each stage's MMAs as soon as it has landed (K = 16 per MMA: 32 B along the swizzled row)
+            bool ok = true;
+            for (int st = 0; st < nst && ok; st++) {
+                const uint32_t a_s = sbase + (uint32_t)st * P.stage_bytes, b_s = a_s + a_bytes;
+                if (!tc_wait(tc_smem(&s_lbar[st]), round & 1u)) {
+                    ok = false;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 #pragma unroll
-                for (int kk = 0; kk < kTcK / 16; kk++) {  // K = 16 per MMA: two core matrices along K
-                    const uint64_t ad = tc_desc(a_s + 256u * kk, 128u, 1024u);
-                    const uint64_t bd = tc_desc(b_s + 256u * kk, 128u, 1024u);
+                for (int kk = 0; kk < kTcK / 16; kk++) {
+                    const uint64_t ad = tc_desc_sw128(a_s + 32u * kk);
+                    const uint64_t bd = tc_desc_sw128(b_s + 32u * kk);
                     const uint32_t acc = accumulate ? 1u : 0u;
                     asm volatile(
                         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -148,20 +172,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const TcParams P) {
                     accumulate = true;
                 }
             }
+            if (!ok) s_fail = 1;
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                          : "memory");
         }
         // the stage buffers are reused (and the accumulator read) only after these MMAs finished
-        if (!tc_wait(mbar, phase)) s_fail = 1;
-        phase ^= 1u;
+        if (!tc_wait(mbar, round & 1u)) s_fail = 1;
         __syncthreads();
+        if (s_fail) break;
     }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-    // partial tile -> shared memory [row][n_pad + 1] (padded rows: conflict-free)
+    // The 8 partial tiles of the cluster are added by the rank that owns the rows
+    // (rank q owns rows [16 q, 16 q + 16)), in rank order (deterministic).  Each CTA
+    // first writes its accumulator to shared memory, [row][ldp] fp32.
     float* part = reinterpret_cast<float*>(smem);
-    const int ldp = n_pad + 1;
     const int row = 32 * warp + lane;
+    const int n_valid = min(n_pad, P.T - P.t_base);
+    const bool bulk = n_pad <= kTcBulkCols;
+    const int ldp = bulk ? n_pad : n_pad + 4;  // bulk: rows contiguous; pull: 16-byte aligned, padded
     for (int c0 = 0; c0 < n_pad; c0 += 16) {
         uint32_t v[16];
         asm volatile(
@@ -171,26 +200,80 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const TcParams P) {
             : "r"(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-        for (int i = 0; i < 16; i++) part[row * ldp + c0 + i] = __uint_as_float(v[i]);
+        for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(part + row * ldp + c0 + i) =
+                make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                            __uint_as_float(v[i + 3]));
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    // rank q of the cluster adds the 8 partials of rows [16 q, 16 q + 16) in rank order
-    const int n_valid = min(n_pad, P.T - P.t_base);
-    for (int e = tid; e < 16 * n_valid; e += kTcThreads) {
-        const int rr = 16 * (int)rank + (e & 15), n = e >> 4;
-        const uint32_t local = tc_smem(part + rr * ldp + n);
-        float s = 0.0f;
-        for (uint32_t q = 0; q < kTcCluster; q++) {
-            uint32_t remote;
-            float v;
-            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(q));
-            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-            s += v;
+    if (bulk) {
+        // Each rank's 16 rows (one contiguous 16 x n_pad block) go to that rank's
+        // receive slice [this rank] by one bulk copy, completing on its mbarrier; no
+        // cluster barrier: the receive slices are memory no one else uses.
+        float* recv = reinterpret_cast<float*>(smem + P.recv_off);  // [source rank][16][n_pad]
+        const uint32_t slice = 16u * (uint32_t)n_pad * 4u;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // this thread's writes -> the copies' reads
+        // every CTA of the cluster has initialised (and armed) its receive mbarrier
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        __syncthreads();  // the partial tile is written
+        if (tid == 0) {
+            for (uint32_t q = 0; q < kTcCluster; q++) {
+                uint32_t dst, bar;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                             : "=r"(dst)
+                             : "r"(tc_smem(recv + (size_t)rank * 16 * n_pad)), "r"(q));
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(bar) : "r"(tc_smem(&s_rbar)), "r"(q));
+                asm volatile(
+                    "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                        dst),
+                    "r"(tc_smem(part + (size_t)q * 16 * n_pad)), "r"(slice), "r"(bar)
+                    : "memory");
+            }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the sources are read
         }
-        P.Z[(size_t)(P.t_base + n) * P.r + m0 + rr] = s;
+        if (!tc_wait(tc_smem(&s_rbar), 0)) s_fail = 1;  // this rank's 8 slices have arrived
+        for (int e = tid; e < 16 * n_valid; e += kTcThreads) {
+            const int rr = e & 15, n = e >> 4;  // consecutive threads: consecutive rows of one token
+            float sum = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kTcCluster; q++) sum += recv[((size_t)q * 16 + rr) * n_pad + n];
+            P.Z[(size_t)(P.t_base + n) * P.r + m0 + 16 * (int)rank + rr] = sum;
+        }
+    } else {
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // the start-up arrival
+        asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        // pull: 4 columns at a time, the 8 remote 16-byte loads of an element group
+        // issued back to back (their latencies overlap), then added in rank order
+        const int ngrp = (n_valid + 3) / 4;
+        for (int e = tid; e < 16 * ngrp; e += kTcThreads) {
+            const int rr = 16 * (int)rank + (e & 15), cg = e >> 4;
+            const uint32_t local = tc_smem(part + rr * ldp + 4 * cg);
+            float4 v[kTcCluster];
+#pragma unroll
+            for (int q = 0; q < kTcCluster; q++) {
+                uint32_t remote;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(q));
+                asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(v[q].x), "=f"(v[q].y), "=f"(v[q].z), "=f"(v[q].w)
+                             : "r"(remote));
+            }
+            float4 sum = v[0];
+#pragma unroll
+            for (int q = 1; q < kTcCluster; q++) {
+                sum.x += v[q].x;
+                sum.y += v[q].y;
+                sum.z += v[q].z;
+                sum.w += v[q].w;
+            }
+            const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                if (4 * cg + j < n_valid) P.Z[(size_t)(P.t_base + 4 * cg + j) * P.r + m0 + rr] = sv[j];
+        }
     }
-    asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // no CTA leaves while another may still read its shared memory (the pull)
+    if (!bulk) asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
     if (s_fail && tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (warp == 0)
@@ -202,8 +285,40 @@ bool proj_tc_supported(int T, int d_in, int r) {
     return T >= 8 && r % kTcM == 0 && d_in % (kTcK * kTcCluster) == 0;
 }
 
+// A 2-D fp16 tensor map over rows x d_in (row-major), boxes of 64 K-elements x
+// box_rows rows in the 128-byte swizzle; rows past the end read as zeros.
+static int tc_tensor_map(CUtensorMap* map, const uint16_t* base, int d_in, int rows, int box_rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    // The driver function comes through the runtime's entry-point query, so the
+    // library does not link libcuda (it loads on a machine without a GPU driver).
+    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static std::atomic<EncodeFn> s_encode{nullptr};
+    EncodeFn encode = s_encode.load(std::memory_order_acquire);
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return set_cuda_error(e);
+        if (q != cudaDriverEntryPointSuccess || !fn) return set_cuda_error(cudaErrorSymbolNotFound);
+        encode = reinterpret_cast<EncodeFn>(fn);
+        s_encode.store(encode, std::memory_order_release);
+    }
+    const CUresult rc = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)base, dims, strides, box, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return rc == CUDA_SUCCESS ? BITSMOE_OK : set_cuda_error(cudaErrorInvalidValue);
+}
+
 int launch_proj_tc(const uint16_t* phi_t, const uint16_t* X, float* Z, int T, int d_in, int r, int32_t* status,
                    cudaStream_t s) {
+    CUtensorMap tmA;
+    int rc = tc_tensor_map(&tmA, phi_t, d_in, r, kTcM);
+    if (rc) return rc;
     for (int t_base = 0; t_base < T; t_base += 256) {
         TcParams P{};
         P.phi_t = phi_t;
@@ -216,9 +331,14 @@ int launch_proj_tc(const uint16_t* phi_t, const uint16_t* X, float* Z, int T, in
         P.t_base = t_base;
         P.n_pad = (int)roundup((uint64_t)std::min(256, T - t_base), 16);
         P.k_per_cta = d_in / kTcCluster;
-        P.stage_bytes = (uint32_t)(kTcM * kTcK * 2 + P.n_pad * kTcK * 2);
-        const size_t smem = std::max<size_t>((size_t)kTcMaxStages * P.stage_bytes,
-                                             (size_t)kTcM * (P.n_pad + 1) * 4) + 1024;
+        P.stage_bytes = (uint32_t)(kTcM * kTcK * 2 + P.n_pad * kTcK * 2);  // a multiple of 1024 (n_pad % 16 == 0)
+        CUtensorMap tmB;
+        rc = tc_tensor_map(&tmB, X, d_in, T, P.n_pad);
+        if (rc) return rc;
+        // stages (later the partial tile), then the receive slices of the bulk reduction
+        const size_t tile_bytes = std::max<size_t>((size_t)kTcMaxStages * P.stage_bytes, (size_t)kTcM * (P.n_pad + 4) * 4);
+        P.recv_off = (uint32_t)roundup(tile_bytes, 128);
+        const size_t smem = P.recv_off + (P.n_pad <= kTcBulkCols ? (size_t)kTcCluster * 16 * P.n_pad * 4 : 0) + 1024;
         cudaError_t e = cudaFuncSetAttribute(k_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return set_cuda_error(e);
         cudaLaunchConfig_t cfg{};
@@ -233,7 +353,7 @@ int launch_proj_tc(const uint16_t* phi_t, const uint16_t* X, float* Z, int T, in
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, k_proj_tc, P);
+        e = cudaLaunchKernelEx(&cfg, k_proj_tc, P, tmA, tmB);
         if (e != cudaSuccess) return set_cuda_error(e);
     }
     return BITSMOE_OK;
