@@ -83,8 +83,10 @@ def lib():
         L.orc_shared_proj.restype = None
         L.orc_expert_forward.argtypes = [c_u8p, ctypes.c_uint64, c_f64p, c_i32p, c_f32p, ctypes.c_int,
                                          ctypes.c_int, c_f64p, c_f64p, c_i32p]
+        L.orc_ffn_down.argtypes = [c_f64p, c_f64p, c_u16p, c_i32p, c_f32p, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, c_f64p, c_i32p]
         for f in ("orc_compute_scales", "orc_pack", "orc_blob_parse", "orc_unpack", "orc_dequant_expert",
-                  "orc_expert_forward"):
+                  "orc_expert_forward", "orc_ffn_down"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -248,6 +250,37 @@ def layer_forward(blob_gate, blob_up, phi_t_gate_bits, phi_t_up_bits, x_bits, id
         Ye, Ys, st = expert_forward(blob, Z, ids, gate_w, want_experts)
         out[name] = {"Z": Z, "Y_experts": Ye, "Y_sum": Ys, "status": st}
     return out
+
+
+def ffn_down(Y_gate: np.ndarray, Y_up: np.ndarray, w_down_bits: np.ndarray, ids: np.ndarray, gate_w: np.ndarray):
+    """Expert FFN output after the gate and up projections (the pages stop at
+    gate/up; this is the usual gated expert with a dense fp16 down projection):
+    out[t] = sum_s g[t][s] Wd[e] (SiLU(Y_gate[t][s]) * Y_up[t][s]), e = ids[t][s].
+
+    Y_gate, Y_up [T][top_k][d_ff] (fp64), w_down_bits [E][d_model][d_ff] fp16 bits,
+    ids [T][top_k], gate_w [T][top_k].  Returns (out [T][d_model] fp64, status)."""
+    Yg = _c(Y_gate, np.float64)
+    Yu = _c(Y_up, np.float64)
+    W = _c(w_down_bits, np.uint16)
+    ids = _c(ids, np.int32)
+    g = _c(gate_w, np.float32)
+    T, top_k = ids.shape
+    E, d_model, d_ff = W.shape
+    assert Yg.shape == (T, top_k, d_ff) and Yu.shape == Yg.shape and g.shape == ids.shape
+    out = np.zeros((T, d_model), np.float64)
+    st = ctypes.c_int32(0)
+    _check(lib().orc_ffn_down(_p(Yg, ctypes.c_double), _p(Yu, ctypes.c_double), _p(W, ctypes.c_uint16),
+                              _p(ids, ctypes.c_int32), _p(g, ctypes.c_float), T, top_k, E, d_model, d_ff,
+                              _p(out, ctypes.c_double), ctypes.byref(st)), "ffn_down")
+    return out, int(st.value)
+
+
+def moe_ffn_forward(blob_gate, blob_up, phi_t_gate_bits, phi_t_up_bits, x_bits, ids, gate_w, w_down_bits):
+    """The whole expert FFN of one layer: the gate and up projections in spectral
+    form (layer_forward), then SiLU(gate) * up and the dense down projection."""
+    lf = layer_forward(blob_gate, blob_up, phi_t_gate_bits, phi_t_up_bits, x_bits, ids, gate_w, True)
+    out, st = ffn_down(lf["gate"]["Y_experts"], lf["up"]["Y_experts"], w_down_bits, ids, gate_w)
+    return out, lf["gate"]["status"] | lf["up"]["status"] | st
 
 
 # ---------------------------------------------------------------------------

@@ -584,3 +584,51 @@ int orc_expert_forward(const uint8_t *blob, uint64_t bytes, const double *Z, con
     if (status) *status |= st;
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Expert FFN output after the gate and up projections.                      */
+/* ------------------------------------------------------------------------- */
+
+/* The pages decompose only an expert's gate and up projections (Methodology:
+ * the stacked gate/up matrices) and say nothing of what follows them.  This
+ * is the usual gated MoE expert, with a dense fp16 down projection per
+ * expert, in fp64 from the gate and up outputs:
+ *   h[t][s][m] = SiLU(Yg[t][s][m]) * Yu[t][s][m],   SiLU(v) = v / (1 + e^(-v))
+ *   out[t][i]  = sum_s g[t][s] * sum_m Wd[e][i][m] * h[t][s][m],  e = ids[t][s]
+ * Yg, Yu are [T][top_k][d_ff] (the per-slot expert outputs of the gate and up
+ * projections), Wd is [E][d_model][d_ff] fp16 bits (row i of expert e holds
+ * the weights of output i), out is [T][d_model].  An id outside [0, E)
+ * contributes nothing and sets ORC_ST_BADEXPERT. */
+static double orc_silu(double v) { return v / (1.0 + exp(-v)); }
+
+int orc_ffn_down(const double *Yg, const double *Yu, const uint16_t *w_down, const int32_t *ids, const float *g,
+                 int T, int top_k, int E, int d_model, int d_ff, double *out, int32_t *status) {
+    if (T < 0 || top_k < 1 || E < 1 || d_model < 1 || d_ff < 1) return ORC_EINVAL;
+    if (T > 0 && (!Yg || !Yu || !w_down || !ids || !g || !out)) return ORC_EINVAL;
+    int32_t st = 0;
+    double *h = (double *)malloc(sizeof(double) * (size_t)d_ff);
+    if (!h) return ORC_EINVAL;
+    for (int t = 0; t < T; t++) {
+        double *o = out + (size_t)t * d_model;
+        for (int i = 0; i < d_model; i++) o[i] = 0.0;
+        for (int s = 0; s < top_k; s++) {
+            const size_t q = (size_t)t * top_k + s;
+            const int e = ids[q];
+            if (e < 0 || e >= E) {
+                st |= ORC_ST_BADEXPERT;
+                continue;
+            }
+            for (int m = 0; m < d_ff; m++) h[m] = orc_silu(Yg[q * d_ff + m]) * Yu[q * d_ff + m];
+            const double gw = (double)g[q];
+            for (int i = 0; i < d_model; i++) {
+                const uint16_t *row = w_down + ((size_t)e * d_model + i) * d_ff;
+                double acc = 0.0;
+                for (int m = 0; m < d_ff; m++) acc += orc_f16_to_f64(row[m]) * h[m];
+                o[i] += gw * acc;
+            }
+        }
+    }
+    free(h);
+    if (status) *status |= st;
+    return ORC_OK;
+}

@@ -503,3 +503,98 @@ def test_synth_tiny_layer_shapes():
         order = np.argsort(-L["gate"]["amps"][e].numpy(), kind="stable")
         assert w[e].numpy()[order[:8]].tolist() == [16] * 8
     assert L["ids"].shape == (4, 2) and np.allclose(L["gate_w"].sum(1).numpy(), 1, atol=1e-6)
+
+
+# --------------------------------------------------------------------------
+# expert FFN output: SiLU(gate) * up, then the dense down projection
+# --------------------------------------------------------------------------
+
+def test_ffn_silu_closed_forms(orc):
+    """With an identity down matrix and g = 1 the output is SiLU(y_g) * y_u per
+    column.  The logistic function has closed forms at ln 3 (3/4), -ln 3 (1/4)
+    and 0 (1/2); far out it saturates to 1 (v = 40: v exactly) and to 0 without
+    an overflow NaN (v = -800).  Gate and up enter asymmetrically, so swapping
+    them fails the first column."""
+    ln3 = np.log(3.0)
+    W = np.eye(6, dtype=np.float16).view(np.uint16)[None]
+    Yg = np.array([[[ln3, -ln3, 0.0, 40.0, -800.0, 1.0]]])
+    Yu = np.array([[[1.0, 2.0, -3.0, 0.5, 7.0, ln3]]])
+    out, st = orc.ffn_down(Yg, Yu, W, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32))
+    assert st == 0
+    expect = np.array([0.75 * ln3, -0.5 * ln3, 0.0, 20.0, 0.0, ln3 / (1 + np.exp(-1.0))])
+    assert np.allclose(out[0, :4], expect[:4], rtol=1e-15, atol=0)
+    assert out[0, 4] == 0.0 and np.isfinite(out).all()
+    assert abs(out[0, 5] - expect[5]) <= 1e-15 * abs(expect[5])
+
+
+def _dense_gate_up(orc, blob, e, Phi):
+    Wd, a = orc.dequant_expert(blob, e)
+    return (Wd.T * a) @ Phi.T  # [d_out][d_in]
+
+
+def test_ffn_matches_dense_expert_brute_force(orc):
+    """The oracle's whole expert FFN (spectral gate/up, then SiLU(gate) * up and the
+    down projection) equals the textbook dense gated expert built from the same
+    dequantised factors: out = sum_s g_s Wd_e (silu(Wg_e x) * (Wu_e x)), with
+    SiLU from scipy's logistic function and numpy matmuls, on a non-square case
+    (d_model = 24 != d_ff = 16) so a transposed operand cannot pass."""
+    from scipy.special import expit
+    rng = np.random.default_rng(61)
+    E, r, d_ff, d_model, T = 3, 24, 16, 24, 3
+    blobs = {}
+    for name in ("gate", "up"):
+        comps, widths, amps = _random_case(rng, E, r, d_ff)
+        scales, _ = orc.compute_scales(comps, widths)
+        blobs[name], _ = orc.pack(comps, widths, scales, amps)
+    phi_t = {n: rng.standard_normal((r, d_model)).astype(np.float16) for n in ("gate", "up")}
+    w_down = (rng.standard_normal((E, d_model, d_ff)) / 4).astype(np.float16)
+    x = rng.standard_normal((T, d_model)).astype(np.float16)
+    ids = np.array([[0, 2], [1, 1], [2, 0]], np.int32)
+    g = np.array([[0.7, 0.3], [0.5, 0.5], [0.1, 0.9]], np.float32)
+    out, st = orc.moe_ffn_forward(blobs["gate"], blobs["up"], phi_t["gate"].view(np.uint16),
+                                  phi_t["up"].view(np.uint16), x.view(np.uint16), ids, g, w_down.view(np.uint16))
+    assert st == 0 and out.shape == (T, d_model)
+    X = x.astype(np.float64)
+    for t in range(T):
+        ref = np.zeros(d_model)
+        for s in range(ids.shape[1]):
+            e = int(ids[t, s])
+            yg = _dense_gate_up(orc, blobs["gate"], e, phi_t["gate"].astype(np.float64).T) @ X[t]
+            yu = _dense_gate_up(orc, blobs["up"], e, phi_t["up"].astype(np.float64).T) @ X[t]
+            h = yg * expit(yg) * yu
+            ref += float(g[t, s]) * (w_down[e].astype(np.float64) @ h)
+        assert np.max(np.abs(out[t] - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_ffn_routing_invariants(orc):
+    """Permuting the top-k slots keeps the output; it is linear in g and in the
+    down matrix; a token alone equals the same token in a batch; an id out of
+    range drops its slot and sets the status bit; T = 0 gives an empty output."""
+    rng = np.random.default_rng(71)
+    E, d_model, d_ff, T, K = 4, 10, 12, 3, 3
+    W = (rng.standard_normal((E, d_model, d_ff)) / 3).astype(np.float16)
+    Yg = rng.standard_normal((T, K, d_ff)) * 2
+    Yu = rng.standard_normal((T, K, d_ff))
+    ids = np.array([[0, 3, 1], [2, 2, 0], [3, 1, 0]], np.int32)
+    g = rng.uniform(0.1, 1, (T, K)).astype(np.float32)
+    out, st = orc.ffn_down(Yg, Yu, W.view(np.uint16), ids, g)
+    assert st == 0
+    perm = [2, 0, 1]
+    out2, _ = orc.ffn_down(Yg[:, perm], Yu[:, perm], W.view(np.uint16), ids[:, perm], g[:, perm])
+    assert np.allclose(out2, out, rtol=1e-14, atol=1e-14)
+    out3, _ = orc.ffn_down(Yg, Yu, W.view(np.uint16), ids, (2 * g).astype(np.float32))
+    assert np.allclose(out3, 2 * out, rtol=1e-14, atol=1e-14)
+    W2 = (2 * W.astype(np.float32)).astype(np.float16)  # exact: a power-of-two scaling
+    out4, _ = orc.ffn_down(Yg, Yu, W2.view(np.uint16), ids, g)
+    assert np.array_equal(out4, 2 * out)
+    out1, _ = orc.ffn_down(Yg[1:2], Yu[1:2], W.view(np.uint16), ids[1:2], g[1:2])
+    assert np.array_equal(out1[0], out[1])
+    bad = ids.copy()
+    bad[0, 1] = E
+    out5, st5 = orc.ffn_down(Yg, Yu, W.view(np.uint16), bad, g)
+    assert st5 == orc.ST_BADEXPERT
+    keep = [0, 2]
+    out6, _ = orc.ffn_down(Yg[:1, keep], Yu[:1, keep], W.view(np.uint16), ids[:1, keep], g[:1, keep])
+    assert np.allclose(out5[0], out6[0], rtol=1e-14, atol=1e-14) and np.array_equal(out5[1:], out[1:])
+    out0, st0 = orc.ffn_down(Yg[:0], Yu[:0], W.view(np.uint16), ids[:0], g[:0])
+    assert out0.shape == (0, d_model) and st0 == 0
