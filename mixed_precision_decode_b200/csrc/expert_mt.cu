@@ -16,7 +16,8 @@
 // four of the expert's tokens with one bulk copy each.  Each warp takes a contiguous
 // range of the expert's member words (balanced by plane words) and, per word,
 // builds in its own 2 KB of shared memory the word's 16-entry subset-sum
-// tables whose entries are token PAIRS (float2), with shuffles, then looks up
+// tables whose entries are token PAIRS (float2), from broadcast 16-byte loads
+// of the staged c rows, then looks up
 // every plane word of the member word for every tile: one conflict-free 8-byte
 // shared load per 4-member nibble and two tokens, a lane per row.  The loop
 // needs no CTA barrier; the warps' partial sums are added in warp order at the
@@ -99,6 +100,26 @@ __device__ __forceinline__ float mt_lds1(uint32_t addr) {
     float v;
     asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
     return v;
+}
+
+// Warp 0 (every lane): records the token group's pairs (lane u holds the pair of
+// token u, or -1 past the group's nt tokens) and their zero-point totals, and
+// issues one bulk copy of each pair's c row into row u of s_c, all on one phase
+// of bar.  In the checked build a copy that would leave its buffer is skipped
+// and not counted in the phase's bytes.
+__device__ __forceinline__ void mt_issue_group(const MtParams& P, int pr, int nt, uint32_t members, int lane,
+                                               int* s_pair, float* s_zp, float* s_c, uint64_t* bar) {
+    const bool ok = lane < nt && pr >= 0 && members > 0 &&
+                    in_bounds((uint64_t)(lane + 1) * members - 1, P.c_floats, P.status) &&
+                    in_bounds((uint64_t)pr, (uint64_t)P.n_pairs, P.status);
+    const uint32_t okm = __ballot_sync(0xffffffffu, ok);
+    if (lane == 0) mt_expect_tx(bar, 4u * members * (uint32_t)__popc(okm));
+    __syncwarp();
+    if (ok) mt_bulk(s_c + (size_t)lane * members, P.rw.cvals + (size_t)pr * P.rw.ldc, 4u * members, bar);
+    if (lane < kMtTok) {
+        s_pair[lane] = lane < nt ? pr : -1;
+        s_zp[lane] = ok ? P.rw.zp[pr] : 0.0f;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -217,10 +238,23 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     const uint32_t my_tab_s = tab_s + 2048u * (uint32_t)warp;
     float* s_part = reinterpret_cast<float*>(s_tab);  // reused after the lookups: [warp][tile][32][kMtTok]
 
-    // ---- stage this CTA's rows of every plane word of the expert ----
+    // ---- warp 0: the first token group's c rows are requested first (the pair ids
+    // load while lane 0 reads the directory), then lane 0 lays out the expert ----
     if (warp == 0) {
+        const int nt0 = min(kMtTok, p1 - p0);
+        const int pr0 = lane < nt0 ? P.rw.pairs[p0 + lane] : -1;
+        DirEntry d;
+        uint32_t members0 = 0;
         if (lane == 0) {
-            const DirEntry d = read_dir(P.blob, e);
+            d = read_dir(P.blob, e);
+            for (int g = 0; g < kNumGroups; g++) members0 += (uint32_t)group_members_padded(group_width(g), d.count[g]);
+            s_fail = 0;
+            mt_mbar_init(&s_cbar);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        members0 = __shfl_sync(0xffffffffu, members0, 0);
+        mt_issue_group(P, pr0, nt0, members0, lane, s_pair, s_zp, s_c, &s_cbar);
+        if (lane == 0) {
             uint32_t so = 0, co = 0, pw = 0, pwords = 0;
             for (int g = 0; g < kNumGroups; g++) {
                 const int b = group_width(g);
@@ -252,9 +286,6 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                 }
             }
             while (wv < kMtWarps) s_wbeg[++wv] = (int)word;
-            s_fail = 0;
-            mt_mbar_init(&s_cbar);
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
             s_ex.plane_words = pwords;
         }
     }
@@ -293,20 +324,16 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
     for (int pq = p0; pq < p1; pq += kMtTok) {
         const int nt = min(kMtTok, p1 - pq);
         const int npairs = (nt + 1) / 2;  // token pairs with a routed token (the second is skipped if empty)
-        __syncthreads();  // the previous group's c rows and partial sums are no longer read
-        // ---- the c rows of this group's tokens (one bulk copy each) ----
-        if (tid == 0) {
-            mt_expect_tx(&s_cbar, 4u * members * (uint32_t)nt);
-            for (int u = 0; u < kMtTok; u++) {
-                const int pr = u < nt ? P.rw.pairs[pq + u] : -1;
-                s_pair[u] = pr;
-                s_zp[u] = pr >= 0 ? P.rw.zp[pr] : 0.0f;
-                if (pr >= 0 && members > 0 && in_bounds((uint64_t)(u + 1) * members - 1, P.c_floats, P.status) &&
-                    in_bounds(pr, (uint64_t)P.n_pairs, P.status))
-                    mt_bulk(s_c + (size_t)u * members, P.rw.cvals + (size_t)pr * P.rw.ldc, 4u * members, &s_cbar);
+        // ---- the c rows of this group's tokens (one bulk copy each; the first
+        // group's went out before the staging) ----
+        if (pq != p0) {
+            __syncthreads();  // the previous group's c rows and partial sums are no longer read
+            if (warp == 0) {
+                const int pr = lane < nt ? P.rw.pairs[pq + lane] : -1;
+                mt_issue_group(P, pr, nt, members, lane, s_pair, s_zp, s_c, &s_cbar);
             }
-            if (!mt_mbar_wait(&s_cbar, cphase)) s_fail = 1;
         }
+        if (tid == 0 && !mt_mbar_wait(&s_cbar, cphase)) s_fail = 1;
         cphase ^= 1u;
         if (pq == p0) asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's pieces of the planes
         __syncthreads();
@@ -332,11 +359,10 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
             }
             const int b = group_width(g), w = wi - wg0;
             const uint32_t W = s_ex.W[g];
-            const float* cg = s_c + s_ex.c_off[g];
-            const uint32_t m = 32u * (uint32_t)w + (uint32_t)lane;
-            float c[kMtTok];
-#pragma unroll
-            for (int u = 0; u < kMtTok; u++) c[u] = u < nt ? cg[(size_t)u * members + m] : 0.0f;
+            // this word's c values of token 0; token u's are members floats further on.  A
+            // table's four members are one 16-byte load per token, shared by the 16 lanes
+            // that build the table (a broadcast): no shuffles
+            const float* cw = s_c + s_ex.c_off[g] + 32u * (uint32_t)w;
             __syncwarp();  // the previous word's lookups are done with the tables
             if (nt == 1) {
                 // one token: float tables (8 x 16 entries, 512 B), one 4-byte lookup per
@@ -346,12 +372,9 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
 #pragma unroll
                 for (int qq = 0; qq < 4; qq++) {
                     const int tb = (lane >> 4) + 2 * qq;
-                    const float x0 = __shfl_sync(0xffffffffu, c[0], 4 * tb);
-                    const float x1 = __shfl_sync(0xffffffffu, c[0], 4 * tb + 1);
-                    const float x2 = __shfl_sync(0xffffffffu, c[0], 4 * tb + 2);
-                    const float x3 = __shfl_sync(0xffffffffu, c[0], 4 * tb + 3);
-                    tab1[tb * 16 + e1] =
-                        ((e1 & 1 ? x0 : 0.0f) + (e1 & 2 ? x1 : 0.0f)) + ((e1 & 4 ? x2 : 0.0f) + (e1 & 8 ? x3 : 0.0f));
+                    const float4 xv = *reinterpret_cast<const float4*>(cw + 4 * tb);
+                    tab1[tb * 16 + e1] = ((e1 & 1 ? xv.x : 0.0f) + (e1 & 2 ? xv.y : 0.0f)) +
+                                         ((e1 & 4 ? xv.z : 0.0f) + (e1 & 8 ? xv.w : 0.0f));
                 }
                 __syncwarp();
                 const uint32_t* stg1 = s_stage + s_ex.stage_off[g] + (uint32_t)w * (uint32_t)ntl * 32u + (uint32_t)lane;
@@ -375,25 +398,23 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
                 continue;
             }
             // entry en of table tb of pair pr = the sums of c over the set bits of en
-            // (members 4 tb .. 4 tb + 3) for tokens 2 pr and 2 pr + 1
+            // (members 4 tb .. 4 tb + 3) for tokens 2 pr and 2 pr + 1; a token past the
+            // group's last (its c row holds an earlier group's values) counts as 0
             const int en = lane & 15;
 #pragma unroll
             for (int pr = 0; pr < kMtPairs; pr++) {
                 if (pr >= npairs) break;
+                const bool has_y = 2 * pr + 1 < nt;
+                const float* cx = cw + (size_t)(2 * pr) * members;
 #pragma unroll
                 for (int qq = 0; qq < 4; qq++) {
                     const int tb = (lane >> 4) + 2 * qq;
-                    const float x0 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb);
-                    const float x1 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb + 1);
-                    const float x2 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb + 2);
-                    const float x3 = __shfl_sync(0xffffffffu, c[2 * pr], 4 * tb + 3);
-                    const float y0 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb);
-                    const float y1 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb + 1);
-                    const float y2 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb + 2);
-                    const float y3 = __shfl_sync(0xffffffffu, c[2 * pr + 1], 4 * tb + 3);
+                    const float4 xv = *reinterpret_cast<const float4*>(cx + 4 * tb);
+                    float4 yv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (has_y) yv = *reinterpret_cast<const float4*>(cx + members + 4 * tb);
                     float2 v;
-                    v.x = ((en & 1 ? x0 : 0.0f) + (en & 2 ? x1 : 0.0f)) + ((en & 4 ? x2 : 0.0f) + (en & 8 ? x3 : 0.0f));
-                    v.y = ((en & 1 ? y0 : 0.0f) + (en & 2 ? y1 : 0.0f)) + ((en & 4 ? y2 : 0.0f) + (en & 8 ? y3 : 0.0f));
+                    v.x = ((en & 1 ? xv.x : 0.0f) + (en & 2 ? xv.y : 0.0f)) + ((en & 4 ? xv.z : 0.0f) + (en & 8 ? xv.w : 0.0f));
+                    v.y = ((en & 1 ? yv.x : 0.0f) + (en & 2 ? yv.y : 0.0f)) + ((en & 4 ? yv.z : 0.0f) + (en & 8 ? yv.w : 0.0f));
                     my_tab[(pr * 8 + tb) * 16 + en] = v;
                 }
             }
@@ -485,17 +506,19 @@ __global__ void __launch_bounds__(kMtThreads) k_expert_mt(const MtParams P) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int g_mt_max_smem = 0;
 
 // Floats per c row: every expert's padded members, rounded to 8 (32-byte rows).
 uint32_t cvals_ldc(const bitsmoe_plan* p) { return (uint32_t)roundup(p->max_members_padded, 8); }
 
 int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, const int32_t* ids, int T,
                      const RouteWS& rw, float* Ye, int32_t* status, cudaStream_t s) {
-    if (g_mt_max_smem == 0) {
+    // the current device's shared-memory limit, looked up on every call (a host-side
+    // query; a process may drive devices of different limits)
+    int max_smem = 0;
+    {
         int dev;
         cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&g_mt_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return set_cuda_error(e);
     }
     if (rw.ldc < cvals_ldc(p)) return BITSMOE_EINVAL;
@@ -531,10 +554,10 @@ int launch_expert_mt(const bitsmoe_plan* p, const void* blob, const float* Z, co
     // alignment), which the warps' partial sums reuse at the end
     static_assert(kMtWarps * kMtMaxTiles * 32 * kMtTok * 4 <= kMtWarps * 2048, "partial sums fit the tables");
     const uint64_t fixed = roundup(4ull * kMtTok * p->max_members_padded, 128) + kMtWarps * 2048ull + 1024 + 128;
-    const uint64_t budget = (uint64_t)g_mt_max_smem - 1024;  // static shared memory of the kernel
+    const uint64_t budget = (uint64_t)max_smem - 1024;  // static shared memory of the kernel
     // the most tiles per CTA that still lets two CTAs share an SM (one stages while
     // the other computes); else the most that fit one CTA per SM
-    const uint64_t half = (uint64_t)g_mt_max_smem / 2 - 1024;
+    const uint64_t half = (uint64_t)max_smem / 2 - 1024;
     int tpc = kMtMaxTiles;
     while (tpc > 1 && fixed + 4 * tile_words * tpc > half) tpc /= 2;
     if (fixed + 4 * tile_words * tpc > half) {
