@@ -44,6 +44,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-chained", action="store_true", help="skip the chained-loop measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ffn", action="store_true",
+                    help="time the whole expert FFN step instead (gate/up layer, then SiLU(gate)*up and the dense "
+                         "fp16 down projection), with the down kernel's own roofline")
+    ap.add_argument("--ffn-two-calls", action="store_true",
+                    help="with --ffn: run each step as bitsmoe_layer_forward then bitsmoe_ffn_down")
     ap.add_argument("--clock-window", type=float, default=0.25,
                     help="seconds of untimed replays of the same loop before the timed steps, during which (and "
                          "during the timed steps) the SM clock is sampled")
@@ -648,6 +653,149 @@ def run_ours(args, dist):
         print(json.dumps(line), flush=True)
 
 
+def down_bytes(cfg, ids_step, T) -> dict:
+    """Bytes the down step must move for one layer step: the dense fp16 down matrix
+    [d_in][d_out] of each distinct routed expert, the gate and up expert outputs
+    (fp32, T x top_k x d_out each), the routing and the fp32 output."""
+    import numpy as np
+    experts = np.unique(ids_step.reshape(-1))
+    w = int(len(experts)) * cfg.d_in * cfg.d_out * 2
+    act = 2 * T * cfg.top_k * cfg.d_out * 4 + T * cfg.top_k * 8 + T * cfg.d_in * 4
+    return {"w_down": w, "act": act, "total": w + act}
+
+
+def run_ffn(args, dist):
+    """The whole expert FFN as a decode loop: per step one bitsmoe_ffn_forward call --
+    the spectral gate/up layer (Y_experts of both projections), then SiLU(gate) * up,
+    the dense fp16 down projection and the slot-order routed sum.  The step loop and,
+    separately, a loop of bitsmoe_ffn_down calls alone (the down kernel's own
+    roofline) are graph-replayed over L layer copies."""
+    import torch
+    from mixed_precision_decode_b200 import bitsmoe as B
+    from mixed_precision_decode_b200 import synth
+    from mixed_precision_decode_b200.layer import SpectralMoEFFN
+
+    cfg = synth.CONFIGS[args.config]
+    if args.tokens:
+        cfg = synth.scaled(cfg, tokens=args.tokens)
+    T = cfg.tokens
+    K, W = args.steps, args.warmup
+    G = max(1, min(K, args.graph_steps))
+    L = args.layers
+    dev = torch.device("cuda")
+    wl = Workload(cfg, L, max(G, L), seed_base=10_000 + 1000 * dist.rank)
+    ffns = [SpectralMoEFFN(layer, synth.make_down(cfg, synth.make_generator(20_000 + 1000 * dist.rank + l, dev), dev))
+            for l, layer in enumerate(wl.layers)]
+    bufs = [layer.forward(wl.x[0], wl.ids[0], wl.gw[0], want_experts=True) for layer in wl.layers]
+    outs = [torch.empty((T, cfg.d_in), dtype=torch.float32, device=dev) for _ in range(L)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+
+    n_dws = B.ffn_down_workspace_bytes(ffns[0].dims, T)
+    down_ws = torch.empty(max(n_dws, 256), dtype=torch.uint8, device=dev)
+
+    def down_step(s):
+        l, d = wl.layer_of(s), wl.data_of(s)
+        f = ffns[l]
+        B.ffn_down(f.dims, f.w_down, bufs[l]["Y_experts_gate"], bufs[l]["Y_experts_up"], wl.ids[d], wl.gw[d], T,
+                   outs[l], down_ws, n_dws)
+
+    def ffn_step(s):
+        l, d = wl.layer_of(s), wl.data_of(s)
+        if args.ffn_two_calls:
+            wl.layers[l].forward(wl.x[d], wl.ids[d], wl.gw[d], out=bufs[l], want_experts=True)
+            down_step(s)
+        else:
+            ffns[l].forward(wl.x[d], wl.ids[d], wl.gw[d], out=outs[l], gate_up=bufs[l])
+
+    def graphs_of(fn):
+        for s in range(-W - L, -L):
+            fn(s)
+        torch.cuda.synchronize()
+        def cap(start, n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                for s in range(start, start + n):
+                    fn(s)
+            return g
+        pre = cap(-L, L)
+        gs = [cap(i, min(G, K - i)) for i in range(0, K, G)]
+        pre.replay()
+        torch.cuda.synchronize()
+        return pre, gs
+
+    def timed(pre, gs, clocks=None, n_pre=1, nvtx=None):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        if clocks:
+            clocks.timed_events = (ev0, ev1)
+            clocks.__enter__()
+        for _ in range(n_pre):
+            pre.replay()
+        if clocks:
+            clocks.sample_now()
+        if nvtx:
+            torch.cuda.nvtx.range_push(nvtx)
+        ev0.record(stream)
+        for g in gs:
+            g.replay()
+        ev1.record(stream)
+        if clocks:
+            clocks.sample_now()
+        torch.cuda.synchronize()
+        if nvtx:
+            torch.cuda.nvtx.range_pop()
+        if clocks:
+            clocks.__exit__(None, None, None)
+        dist.barrier()
+        return dist.max(ev0.elapsed_time(ev1))
+
+    pre, gs = graphs_of(down_step)
+    ms_down = timed(pre, gs, n_pre=2, nvtx="timed_down")
+    del pre, gs
+    pre, gs = graphs_of(ffn_step)
+    clocks = ClockSampler(torch.cuda.current_device(), period_s=0.0)
+    ms = timed(pre, gs, clocks, n_pre=max(2, int(args.clock_window * 1e3 / max(1e-3, L * 0.02))), nvtx="timed")
+    del pre, gs
+    value, step_s = weak_scaling_throughput(dist.world, K, T, ms)
+    down_s = ms_down / 1e3 / K
+
+    counts = {}
+    for s in range(K):
+        key = (wl.layer_of(s), wl.data_of(s))
+        counts[key] = counts.get(key, 0) + 1
+    db = {k: sum(down_bytes(cfg, wl.ids[key[1]].cpu().numpy(), T)[k] * n for key, n in counts.items()) / K
+          for k in ("w_down", "act", "total")}
+    gb = sum(algorithmic_bytes(cfg, wl.counts[key[0]], wl.ids[key[1]].cpu().numpy(), T)["total"] * n
+             for key, n in counts.items()) / K
+    peak, peak_kind = load_peak()
+    n_down = B.ffn_down_launches(ffns[0].dims, T)
+    ach = db["total"] / down_s / 1e9
+    line = {
+        "metric": "decode tokens/s, expert FFN: spectral gate/up + SiLU(gate)*up + dense fp16 down projection",
+        "value": value, "unit": "tokens/s", "n_gpus": dist.world, "steps": K, "warmup": W,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded random factors and down weights of the layer's shape)",
+        "config": dict(workload_config(cfg, T, L), down="dense fp16 [E][d_in][d_out] per expert, N(0,1)/sqrt(d_out)"),
+        "roofline": {"bound": "hbm", "kernel": "k_down_t1" if n_down == 1 else "k_route + k_down_mt + k_combine",
+                     "achieved": ach, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
+                     "traffic": None, "algorithmic_bytes_per_launch": db["total"] if n_down == 1 else None,
+                     "algorithmic_bytes_per_step": db["total"], "duration_us": down_s * 1e6,
+                     "how": "the down calls alone, graph-replayed over the layer copies, timed with CUDA events"},
+        "step_roofline": {"achieved": (gb + db["total"]) / step_s / 1e9, "peak": peak,
+                          "frac": (gb + db["total"]) / step_s / 1e9 / peak,
+                          "bytes_per_step": {"gate_up": gb, "down": db["total"]}},
+        "gpu_launches": (B.layer_launches(wl.layers[0].gate.plan, wl.layers[0].up.plan, T) + n_down
+                         if args.ffn_two_calls else ffns[0].launches(T)) * K,
+        "ffn_call": "bitsmoe_layer_forward + bitsmoe_ffn_down" if args.ffn_two_calls else "bitsmoe_ffn_forward",
+        "clocks": dict(clocks.summary(), window="untimed replays of one rotation and the timed region"),
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def kernels_per_step(wl) -> int:
     from mixed_precision_decode_b200 import bitsmoe as B
     L = wl.layers[0]
@@ -776,6 +924,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, dist)
+        elif args.ffn:
+            run_ffn(args, dist)
         else:
             run_ours(args, dist)
     finally:

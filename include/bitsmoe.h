@@ -247,6 +247,70 @@ int bitsmoe_layer_forward_chained(const bitsmoe_proj_io *gate, const bitsmoe_pro
 int bitsmoe_layer_forward_t1_noalloc(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *X,
                                      const int32_t *topk_ids, const float *gate_w, int32_t *status, void *stream);
 
+/* ---- the expert FFN after the gate and up projections ----
+ * The BitsMoE pages decompose an expert's gate and up projections and stop
+ * there.  These calls finish the expert the usual gated way, with a dense fp16
+ * down projection per expert (the pages leave it uncompressed):
+ *   h[t][j][m] = SiLU(Yg[t][j][m]) * Yu[t][j][m],   SiLU(v) = v / (1 + e^-v),
+ *   out[t][i]  = sum_j g[t][j] sum_m Wd[e][i][m] h[t][j][m],   e = topk_ids[t][j],
+ * where Yg, Yu are the Y_experts outputs of the gate and up projections. */
+typedef struct {
+    int32_t d_model;   /* rows of each down matrix: the layer's hidden width (the gate/up d_in), >= 1 */
+    int32_t d_ff;      /* columns: the gate/up projections' d_out; a multiple of 8 */
+    int32_t n_experts; /* E >= 1 */
+    int32_t top_k;     /* experts per token, >= 1 */
+} bitsmoe_ffn_dims;
+
+/* Workspace bytes bitsmoe_ffn_down needs for T tokens (0 when the single-token
+ * kernel applies: T <= 1 and top_k x d_ff fp32 fit one CTA's shared memory). */
+uint64_t bitsmoe_ffn_down_workspace_bytes(const bitsmoe_ffn_dims *dims, int32_t T);
+
+/* Kernels one bitsmoe_ffn_down call launches: 1 on the single-token path, else 3
+ * (routing groups, the experts' rows, the slot-order sum); 0 for T = 0.
+ * Errors: EINVAL. */
+int bitsmoe_ffn_down_launches(const bitsmoe_ffn_dims *dims, int32_t T);
+
+/* SiLU(gate) * up and the down projection of the routed experts, summed per token.
+ *   w_down dev [E][d_model][d_ff] fp16 (16-byte aligned), Y_gate / Y_up dev
+ *   [T][top_k][d_ff] f32 (16-byte aligned), topk_ids dev [T][top_k] int32,
+ *   gate_w dev [T][top_k] f32 (applied as given), out dev [T][d_model] f32,
+ *   workspace dev (>= bitsmoe_ffn_down_workspace_bytes, 256-byte aligned, no
+ *   initialisation needed; may be NULL when that size is 0), status dev or NULL.
+ * A slot whose id is outside [0, E) contributes nothing and sets
+ * BITSMOE_ST_BADEXPERT.  fp32 arithmetic; each token's sum runs in slot order, so
+ * results do not depend on timing.  The single-token kernel is launched with
+ * programmatic dependent launch: it requests its weight rows into L2 before it
+ * waits for the kernel ahead of it in the stream (the layer call that wrote
+ * Y_gate / Y_up), and reads nothing else before that wait.
+ * Errors: EINVAL (dims, NULL or misaligned pointers), ESIZE (workspace), ECUDA. */
+int bitsmoe_ffn_down(const bitsmoe_ffn_dims *dims, const uint16_t *w_down, const float *Y_gate, const float *Y_up,
+                     const int32_t *topk_ids, const float *gate_w, int32_t T, float *out, void *workspace,
+                     uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* Workspace bytes bitsmoe_ffn_forward needs for T tokens: the layer's, then the
+ * down step's (each on a 256-byte boundary). */
+uint64_t bitsmoe_ffn_workspace_bytes(const bitsmoe_plan *gate, const bitsmoe_plan *up, int32_t T);
+
+/* Kernels one bitsmoe_ffn_forward call launches for T tokens: those of
+ * bitsmoe_layer_forward plus those of bitsmoe_ffn_down.  Errors: EINVAL. */
+int bitsmoe_ffn_launches(const bitsmoe_plan *gate, const bitsmoe_plan *up, int32_t T);
+
+/* The whole expert FFN of one layer for T tokens: bitsmoe_layer_forward, then
+ * bitsmoe_ffn_down on the two projections' per-slot outputs.
+ *   gate, up: as in bitsmoe_layer_forward, with Y_experts set in both (16-byte
+ *   aligned; they are the down step's inputs); the plans agree on d_out.
+ *   w_down dev [E][d_in][d_out] fp16, 16-byte aligned (d_model = the plans' d_in,
+ *   d_ff = their d_out, a multiple of 8).  X, topk_ids, gate_w: as in
+ *   bitsmoe_layer_forward.  out dev [T][d_in] f32.
+ *   workspace dev (>= bitsmoe_ffn_workspace_bytes, 256-byte aligned): its head is
+ *   the layer's workspace, with the same rules (zero-filled once before first use,
+ *   calls that share it must not overlap); the down step's part follows it.
+ * On one token the down kernel follows the fused layer kernel by programmatic
+ * dependent launch (see bitsmoe_ffn_down).  Errors: those of the two calls. */
+int bitsmoe_ffn_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *w_down,
+                        const uint16_t *X, const int32_t *topk_ids, const float *gate_w, int32_t T, float *out,
+                        void *workspace, uint64_t workspace_bytes, int32_t *status, void *stream);
+
 /* Waits for `stream`, then copies the device status word to *out_host.
  * Errors: EINVAL, ECUDA. */
 int bitsmoe_read_status(const int32_t *status_dev, void *stream, int32_t *out_host);

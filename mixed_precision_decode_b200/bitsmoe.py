@@ -27,7 +27,9 @@ EXPORTS = (
     "bitsmoe_plan_header_bytes", "bitsmoe_plan_get_dims", "bitsmoe_plan_write_header", "bitsmoe_compute_scales",
     "bitsmoe_pack", "bitsmoe_unpack_q", "bitsmoe_shared_proj", "bitsmoe_expert_workspace_bytes",
     "bitsmoe_expert_forward", "bitsmoe_layer_workspace_bytes", "bitsmoe_layer_launches", "bitsmoe_layer_forward",
-    "bitsmoe_layer_forward_chained", "bitsmoe_layer_forward_t1_noalloc", "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
+    "bitsmoe_layer_forward_chained", "bitsmoe_layer_forward_t1_noalloc", "bitsmoe_ffn_down_workspace_bytes",
+    "bitsmoe_ffn_down_launches", "bitsmoe_ffn_down", "bitsmoe_ffn_workspace_bytes", "bitsmoe_ffn_launches",
+    "bitsmoe_ffn_forward", "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
 )
 
 
@@ -40,6 +42,11 @@ class BitsMoEError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("d_in", ctypes.c_int32), ("d_out", ctypes.c_int32), ("n_experts", ctypes.c_int32),
                 ("rank", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+
+class FfnDims(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32)]
 
 
 class ProjIO(ctypes.Structure):
@@ -81,6 +88,14 @@ def lib() -> ctypes.CDLL:
                                                u64, vp, vp, vp, vp], ctypes.c_int),
             "bitsmoe_layer_forward_t1_noalloc": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, vp,
                                                   vp], ctypes.c_int),
+            "bitsmoe_ffn_down_workspace_bytes": ([ctypes.POINTER(FfnDims), i32], u64),
+            "bitsmoe_ffn_down_launches": ([ctypes.POINTER(FfnDims), i32], ctypes.c_int),
+            "bitsmoe_ffn_down": ([ctypes.POINTER(FfnDims), vp, vp, vp, vp, vp, i32, vp, vp, u64, vp, vp],
+                                 ctypes.c_int),
+            "bitsmoe_ffn_workspace_bytes": ([vp, vp, i32], u64),
+            "bitsmoe_ffn_launches": ([vp, vp, i32], ctypes.c_int),
+            "bitsmoe_ffn_forward": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, vp, i32, vp, vp, u64,
+                                     vp, vp], ctypes.c_int),
             "bitsmoe_read_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "bitsmoe_strerror": ([ctypes.c_int], ctypes.c_char_p),
             "bitsmoe_version": ([], ctypes.c_int),
@@ -236,6 +251,46 @@ def layer_forward_t1_noalloc(gate: ProjIO, up: ProjIO, X, topk_ids, gate_w, stat
     _check(lib().bitsmoe_layer_forward_t1_noalloc(ctypes.byref(gate), ctypes.byref(up), _ptr(X), _ptr(topk_ids),
                                                   _ptr(gate_w), _ptr(status), _stream(stream)),
            "layer_forward_t1_noalloc")
+
+
+def ffn_dims(d_model: int, d_ff: int, n_experts: int, top_k: int) -> FfnDims:
+    return FfnDims(d_model, d_ff, n_experts, top_k)
+
+
+def ffn_down_workspace_bytes(dims: FfnDims, T: int) -> int:
+    return int(lib().bitsmoe_ffn_down_workspace_bytes(ctypes.byref(dims), T))
+
+
+def ffn_down_launches(dims: FfnDims, T: int) -> int:
+    n = int(lib().bitsmoe_ffn_down_launches(ctypes.byref(dims), T))
+    if n < 0:
+        raise BitsMoEError(n, "ffn_down_launches")
+    return n
+
+
+def ffn_down(dims: FfnDims, w_down, Y_gate, Y_up, topk_ids, gate_w, T: int, out, workspace=None,
+             workspace_bytes: int = 0, status=None, stream=None):
+    _check(lib().bitsmoe_ffn_down(ctypes.byref(dims), _ptr(w_down), _ptr(Y_gate), _ptr(Y_up), _ptr(topk_ids),
+                                  _ptr(gate_w), T, _ptr(out), _ptr(workspace), workspace_bytes, _ptr(status),
+                                  _stream(stream)), "ffn_down")
+
+
+def ffn_workspace_bytes(plan_gate: Plan, plan_up: Plan, T: int) -> int:
+    return int(lib().bitsmoe_ffn_workspace_bytes(plan_gate.handle, plan_up.handle, T))
+
+
+def ffn_launches(plan_gate: Plan, plan_up: Plan, T: int) -> int:
+    n = int(lib().bitsmoe_ffn_launches(plan_gate.handle, plan_up.handle, T))
+    if n < 0:
+        raise BitsMoEError(n, "ffn_launches")
+    return n
+
+
+def ffn_forward(gate: ProjIO, up: ProjIO, w_down, X, topk_ids, gate_w, T: int, out, workspace, workspace_bytes: int,
+                status=None, stream=None):
+    _check(lib().bitsmoe_ffn_forward(ctypes.byref(gate), ctypes.byref(up), _ptr(w_down), _ptr(X), _ptr(topk_ids),
+                                     _ptr(gate_w), T, _ptr(out), _ptr(workspace), workspace_bytes, _ptr(status),
+                                     _stream(stream)), "ffn_forward")
 
 
 def read_status(status, stream=None) -> int:

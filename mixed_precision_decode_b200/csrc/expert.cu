@@ -147,6 +147,20 @@ static int launch_route(const bitsmoe_plan* p, const int32_t* ids, int T, const 
     return check_launch();
 }
 
+// Routing groups of npairs (token, slot) pairs and the slot-order routed sum, for
+// the other steps of the library that group tokens by expert (the down projection).
+int launch_route_ids(const int32_t* ids, int npairs, int E, const RouteWS& rw, int32_t* status, cudaStream_t s) {
+    k_route<<<1, kRouteThreads, 0, s>>>(ids, npairs, E, rw, status);
+    return check_launch();
+}
+int launch_combine(const int32_t* ids, const float* gw, float* Ye, float* Ysum, int T, int K, int E, int d_out,
+                   cudaStream_t s) {
+    const uint64_t n = (uint64_t)T * d_out;
+    const unsigned blocks = (unsigned)std::min<uint64_t>((n + 255) / 256, 4096);
+    k_combine<<<blocks, 256, 0, s>>>(ids, gw, Ye, Ysum, T, K, E, d_out);
+    return check_launch();
+}
+
 static uint64_t expert_ws(const bitsmoe_plan* p, int T, bool need_ye, uint8_t* base, RouteWS* rw, float** ye) {
     WsCursor c{base, 0};
     RouteWS r = take_route(c, p->dims.n_experts, T, p->dims.top_k, cvals_ldc(p));
@@ -283,4 +297,42 @@ BITSMOE_API int bitsmoe_layer_forward_chained(const bitsmoe_proj_io* gate, const
     const uint16_t* next[2] = {next_phi_t_gate, next_phi_t_up};
     return layer_forward_impl(gate, up, X, topk_ids, gate_w, T, workspace, workspace_bytes,
                               next_phi_t_gate ? next : nullptr, status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// the whole expert FFN: the layer (gate and up), then the down step
+// ---------------------------------------------------------------------------
+BITSMOE_API uint64_t bitsmoe_ffn_workspace_bytes(const bitsmoe_plan* gate, const bitsmoe_plan* up, int32_t T) {
+    if (!gate || !up || T < 0) return 0;
+    const bitsmoe_ffn_dims d{gate->dims.d_in, gate->dims.d_out, gate->dims.n_experts, gate->dims.top_k};
+    return roundup(bitsmoe_layer_workspace_bytes(gate, up, T), 256) + bitsmoe_ffn_down_workspace_bytes(&d, T);
+}
+
+BITSMOE_API int bitsmoe_ffn_launches(const bitsmoe_plan* gate, const bitsmoe_plan* up, int32_t T) {
+    if (!gate || !up || T < 0) return BITSMOE_EINVAL;
+    const bitsmoe_ffn_dims d{gate->dims.d_in, gate->dims.d_out, gate->dims.n_experts, gate->dims.top_k};
+    const int nl = bitsmoe_layer_launches(gate, up, T), nd = bitsmoe_ffn_down_launches(&d, T);
+    if (nl < 0) return nl;
+    if (nd < 0) return nd;
+    return nl + nd;
+}
+
+BITSMOE_API int bitsmoe_ffn_forward(const bitsmoe_proj_io* gate, const bitsmoe_proj_io* up, const uint16_t* w_down,
+                                    const uint16_t* X, const int32_t* topk_ids, const float* gate_w, int32_t T,
+                                    float* out, void* workspace, uint64_t workspace_bytes, int32_t* status,
+                                    void* stream) {
+    if (!gate || !up || !gate->plan || !up->plan || T < 0) return BITSMOE_EINVAL;
+    const bitsmoe_plan *pg = gate->plan, *pu = up->plan;
+    if (pg->dims.d_out != pu->dims.d_out) return BITSMOE_EINVAL;
+    const bitsmoe_ffn_dims d{pg->dims.d_in, pg->dims.d_out, pg->dims.n_experts, pg->dims.top_k};
+    if (T == 0) return BITSMOE_OK;
+    if (!gate->Y_experts || !up->Y_experts || !w_down || !out || !workspace) return BITSMOE_EINVAL;
+    if ((uintptr_t)w_down % 16 || (uintptr_t)gate->Y_experts % 16 || (uintptr_t)up->Y_experts % 16) return BITSMOE_EINVAL;
+    if (d.d_ff % 8) return BITSMOE_EINVAL;
+    if (workspace_bytes < bitsmoe_ffn_workspace_bytes(pg, pu, T)) return BITSMOE_ESIZE;
+    const uint64_t lw = bitsmoe_layer_workspace_bytes(pg, pu, T), off = roundup(lw, 256);
+    int rc = layer_forward_impl(gate, up, X, topk_ids, gate_w, T, workspace, lw, nullptr, status, stream);
+    if (rc) return rc;
+    return bitsmoe_ffn_down(&d, w_down, gate->Y_experts, up->Y_experts, topk_ids, gate_w, T, out,
+                            (uint8_t*)workspace + off, workspace_bytes - off, status, stream);
 }

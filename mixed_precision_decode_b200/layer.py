@@ -108,3 +108,58 @@ class SpectralMoELayer:
             B.layer_forward_chained(ios[0], ios[1], x, topk_ids, gate_w, T, ws, ws.numel(), next_layer.gate.phi_t,
                                     next_layer.up.phi_t, status, stream)
         return out
+
+
+class SpectralMoEFFN:
+    """A routed expert FFN: the gate and up projections in shared-spectral form
+    (SpectralMoELayer), then SiLU(gate) * up and a dense fp16 down projection per
+    expert, summed over each token's slots with its gate weights -- one
+    bitsmoe_ffn_forward call.
+
+    w_down [E][d_model][d_ff] fp16 on the GPU, d_model = the layer's d_in and
+    d_ff = the gate/up d_out."""
+
+    def __init__(self, layer: SpectralMoELayer, w_down: torch.Tensor):
+        g = layer.gate
+        assert layer.up.d_out == g.d_out
+        assert w_down.dtype == torch.float16 and tuple(w_down.shape) == (g.n_experts, g.d_in, g.d_out)
+        self.layer = layer
+        self.w_down = w_down.contiguous()
+        self.dims = B.ffn_dims(g.d_in, g.d_out, g.n_experts, g.top_k)
+        self._ws = {}
+
+    def workspace(self, T: int) -> torch.Tensor:
+        """The call's workspace for T tokens (the layer's, then the down step's),
+        zero-filled once on first use: its head keeps the fused path's counters."""
+        ws = self._ws.get(T)
+        if ws is None:
+            n = B.ffn_workspace_bytes(self.layer.gate.plan, self.layer.up.plan, T)
+            ws = torch.zeros(max(n, 256), dtype=torch.uint8, device=self.w_down.device)
+            self._ws[T] = ws
+        return ws
+
+    def launches(self, T: int) -> int:
+        """Kernels one forward launches for T tokens (the layer's, then the down step's)."""
+        return B.ffn_launches(self.layer.gate.plan, self.layer.up.plan, T)
+
+    def gate_up_buffers(self, T: int, device) -> dict:
+        """Output buffers of the gate and up projections (routed sums and per-slot outputs)."""
+        out = {}
+        for name, p in (("gate", self.layer.gate), ("up", self.layer.up)):
+            out[f"Y_sum_{name}"] = torch.empty((T, p.d_out), dtype=torch.float32, device=device)
+            out[f"Y_experts_{name}"] = torch.empty((T, p.top_k, p.d_out), dtype=torch.float32, device=device)
+        return out
+
+    def forward(self, x: torch.Tensor, topk_ids: torch.Tensor, gate_w: torch.Tensor, out: torch.Tensor | None = None,
+                gate_up: dict | None = None, status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """x [T][d_in] fp16, topk_ids [T][top_k] int32, gate_w [T][top_k] f32 -> out [T][d_model] f32.
+        gate_up: the gate/up output buffers (gate_up_buffers) to reuse between calls."""
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.dims.d_model), dtype=torch.float32, device=x.device)
+        if gate_up is None:
+            gate_up = self.gate_up_buffers(T, x.device)
+        ios = self.layer._proj_ios(gate_up)
+        ws = self.workspace(T)
+        B.ffn_forward(ios[0], ios[1], self.w_down, x, topk_ids, gate_w, T, out, ws, ws.numel(), status, stream)
+        return out

@@ -120,6 +120,17 @@ def make_projection(cfg: LayerConfig, gen: torch.Generator, device, experts=None
     return {"phi_t": phi_t, "amps": amps, "comps": comps, "widths": widths}
 
 
+def make_down(cfg: LayerConfig, gen: torch.Generator, device) -> torch.Tensor:
+    """Dense down-projection weights of every expert, w_down [E][d_in][d_out] fp16:
+    N(0, 1) / sqrt(d_out) (fan-in scaling), one expert at a time."""
+    E, d_model, d_ff = cfg.n_experts, cfg.d_in, cfg.d_out
+    w = torch.empty((E, d_model, d_ff), dtype=torch.float16, device=device)
+    for e in range(E):
+        w[e] = (torch.randn((d_model, d_ff), generator=gen, device=device, dtype=torch.float32)
+                * d_ff ** -0.5).to(torch.float16)
+    return w
+
+
 def make_routing(cfg: LayerConfig, gen: torch.Generator, device, tokens: int) -> tuple[torch.Tensor, torch.Tensor]:
     """(ids [T][top_k] int32, gate weights [T][top_k] f32)."""
     E, k, T = cfg.n_experts, cfg.top_k, tokens

@@ -161,3 +161,53 @@ def test_workspace_holds_the_multi_token_c_rows(B):
     # each buffer is rounded up to 256 bytes: the growth may fall short by that per buffer
     grow = B.expert_workspace_bytes(plan, 17) - B.expert_workspace_bytes(plan, 3)
     assert grow >= 14 * K * per_pair - 3 * 256
+
+
+def test_ffn_down_argument_checks_and_sizes(B):
+    """The down step's dims, pointer and workspace checks run on the host before any
+    launch; launch counts and workspace sizes follow the two paths."""
+    import ctypes
+    L = B.lib()
+    q = B.ffn_dims(2048, 768, 128, 8)
+    assert B.ffn_down_launches(q, 0) == 0 and B.ffn_down_launches(q, 1) == 1 and B.ffn_down_launches(q, 64) == 3
+    assert B.ffn_down_workspace_bytes(q, 1) == 0
+    n64 = B.ffn_down_workspace_bytes(q, 64)
+    assert n64 >= 64 * 8 * 2048 * 4 + 64 * 8 * 4  # per-pair down rows and the pair lists
+    big = B.ffn_dims(96, 8192, 8, 8)  # top_k x d_ff beyond one CTA: grouped kernels even at T = 1
+    assert B.ffn_down_launches(big, 1) == 3 and B.ffn_down_workspace_bytes(big, 1) > 0
+    bad = B.ffn_dims(64, 12, 4, 2)  # d_ff % 8
+    assert L.bitsmoe_ffn_down_launches(ctypes.byref(bad), 1) == B.EINVAL
+    assert L.bitsmoe_ffn_down(ctypes.byref(bad), 256, 256, 256, 256, 256, 1, 256, None, 0, None, None) == B.EINVAL
+    assert L.bitsmoe_ffn_down(ctypes.byref(q), None, None, None, None, None, 0, None, None, 0, None, None) == B.OK
+    assert L.bitsmoe_ffn_down(ctypes.byref(q), None, 256, 256, 256, 256, 1, 256, None, 0, None, None) == B.EINVAL
+    assert L.bitsmoe_ffn_down(ctypes.byref(q), 256, 0x1004, 256, 256, 256, 1, 256, None, 0, None,
+                              None) == B.EINVAL  # Y_gate misaligned
+    assert L.bitsmoe_ffn_down(ctypes.byref(q), 256, 256, 256, 256, 256, 64, 256, 512, n64 - 1, None,
+                              None) == B.ESIZE
+    assert L.bitsmoe_ffn_down(ctypes.byref(q), 256, 256, 256, 256, 256, 64, 256, 0x1010, n64, None,
+                              None) == B.EINVAL  # workspace not 256-byte aligned
+    assert L.bitsmoe_ffn_down(ctypes.byref(q), 256, 256, 256, 256, 256, -1, 256, None, 0, None, None) == B.EINVAL
+
+
+def test_ffn_forward_argument_checks(B):
+    """The whole-FFN call needs both projections' per-slot outputs and an aligned
+    down matrix; T = 0 is a no-op; the workspace is the layer's plus the down step's."""
+    import ctypes
+    L = B.lib()
+    w = np.zeros((2, 8), np.uint8)
+    w[:, :4] = 2
+    plan = B.pack_plan(16, 8, 2, 8, 1, w)
+    nl, nf = B.layer_workspace_bytes(plan, plan, 3), B.ffn_workspace_bytes(plan, plan, 3)
+    assert nf >= nl + 3 * 1 * 16 * 4
+    assert B.ffn_launches(plan, plan, 1) == B.layer_launches(plan, plan, 1) + 1
+    assert B.ffn_launches(plan, plan, 3) == B.layer_launches(plan, plan, 3) + 3
+    io = B.proj_io(plan, 256, 256, 256, Y_experts=256)
+    io_noy = B.proj_io(plan, 256, 256, 256)
+    args = (256, 256, 256, 256, 3, 256, 512, nf, None, None)
+    assert L.bitsmoe_ffn_forward(ctypes.byref(io), ctypes.byref(io), 256, 256, 256, 256, 0, 256, None, 0, None,
+                                 None) == B.OK
+    assert L.bitsmoe_ffn_forward(ctypes.byref(io), ctypes.byref(io_noy), *args) == B.EINVAL
+    assert L.bitsmoe_ffn_forward(ctypes.byref(io), ctypes.byref(io), 0x1008, 256, 256, 256, 3, 256, 512, nf, None,
+                                 None) == B.EINVAL  # w_down misaligned
+    assert L.bitsmoe_ffn_forward(ctypes.byref(io), ctypes.byref(io), 256, 256, 256, 256, 3, 256, 512, nf - 1, None,
+                                 None) == B.ESIZE
