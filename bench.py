@@ -779,7 +779,8 @@ def run_ffn(args, dist):
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic (seeded random factors and down weights of the layer's shape)",
         "config": dict(workload_config(cfg, T, L), down="dense fp16 [E][d_in][d_out] per expert, N(0,1)/sqrt(d_out)"),
-        "roofline": {"bound": "hbm", "kernel": "k_down_t1" if n_down == 1 else "k_route + k_down_mt + k_combine",
+        "roofline": {"bound": "hbm", "kernel": "k_down_t1" if n_down == 1 else
+                     f"k_route + {'k_down_tc' if cfg.d_out <= 2048 else 'k_down_mt'} + k_combine",
                      "achieved": ach, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": ach / peak,
                      "traffic": None, "algorithmic_bytes_per_launch": db["total"] if n_down == 1 else None,
                      "algorithmic_bytes_per_step": db["total"], "duration_us": down_s * 1e6,

@@ -19,16 +19,18 @@
 //    After the wait it forms h for every slot in shared memory; a warp dots 4 rows
 //    of one slot at a time, lanes on 16-byte chunks, with every load of a step in
 //    flight before its arithmetic.
-//  * Several tokens (k_down_mt): tokens are grouped by expert (the library's
-//    routing groups); a CTA owns (expert, 128 rows; 32 when a row's h needs several
-//    staged column blocks) and reads those rows once for up to 4 of the expert's
-//    tokens per pass, with h staged in shared memory; each warp works on 4 rows x 4
-//    tokens at a time, its first rows loaded before h is formed.  Each (token, slot)
-//    row is written out and the slot-order sum is a second kernel.
+//  * Several tokens: tokens are grouped by expert (the library's routing groups),
+//    one output row is written per routed (token, slot) and the slot-order sum is a
+//    second kernel.  For d_out <= 2048 the rows come from the tensor cores
+//    (k_down_tc, below); otherwise k_down_mt: a CTA owns (expert, 128 rows; 32 when
+//    a row's h needs several staged column blocks) and reads those rows once for up
+//    to 4 of the expert's tokens per pass, with h staged in shared memory; each
+//    warp works on 4 rows x 4 tokens at a time, its first rows loaded before h.
 #include <algorithm>
 #include <atomic>
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace bitsmoe {
 
@@ -346,6 +348,223 @@ __global__ void __launch_bounds__(kDmThreads) k_down_mt(const DownMtParams P) {
 }
 
 // ---------------------------------------------------------------------------
+// several tokens on the tensor cores (d_out of the gate/up projections <= 2048)
+// ---------------------------------------------------------------------------
+// Per routed expert the down step is a dense contraction, out[pair][i] = sum_m
+// Wd[e][i][m] h[pair][m], over the expert's few tokens: one CTA per (expert, 128
+// rows) computes it with tcgen05.mma (kind::f16, fp32 accumulation in tensor
+// memory).  A = 128 rows of Wd[e] (fp16, K-major as stored), streamed by 2-D TMA
+// tiles of 64 K-elements through a ring of 4 stages.  B = 16 rows built in shared
+// memory by the CTA: for up to 8 tokens of the expert, h / s_u split into an fp16
+// high part (rows 0..7) and the fp16 rest (rows 8..15), so that the two columns
+// of a token add up to the product with h to fp32 accuracy; s_u is a power of two
+// that puts the token's largest |h| in [2^14, 2^15), inside fp16's range.
+constexpr int kDcThreads = 128;   // 4 warps: tensor-memory lanes 0..127 = the tile's rows
+constexpr int kDcM = 128;         // rows of an expert's down matrix per tile
+constexpr int kDcK = 64;          // K per stage: one 128-byte swizzled row of fp16
+constexpr int kDcStages = 4;      // ring of A stages
+constexpr int kDcTok = 8;         // tokens per pass
+constexpr int kDcN = 2 * kDcTok;  // B rows: high parts, then low parts
+constexpr int kDcMaxDff = 2048;   // B of every K stage stays resident: 16 x 2048 x 2 = 64 KB
+constexpr uint32_t kDcAStage = kDcM * kDcK * 2;  // 16 KB
+constexpr uint32_t kDcBStage = kDcN * kDcK * 2;  // 2 KB
+constexpr uint32_t kDcTmemCols = 32;             // the smallest allocation; N = 16 columns used
+
+struct DownTcParams {
+    const float* yg;  // [T*K][d_ff]
+    const float* yu;  // [T*K][d_ff]
+    RouteWS rw;       // routing groups
+    float* ydown;     // [T*K][d_model]
+    int32_t* status;
+    int E, d_model, d_ff;
+    int nst;  // K stages: ceil(d_ff / kDcK)
+};
+
+// The 8 values h[m], m = 8c .. 8c+7, of a routed pair (fp32).
+__device__ __forceinline__ void h8_of(const DownTcParams& P, int pair, int c, float (&h)[8]) {
+    const float4* g = reinterpret_cast<const float4*>(P.yg + (size_t)pair * P.d_ff) + 2 * c;
+    const float4* u = reinterpret_cast<const float4*>(P.yu + (size_t)pair * P.d_ff) + 2 * c;
+    const float4 ha = silu_mul(g[0], u[0]), hb = silu_mul(g[1], u[1]);
+    h[0] = ha.x; h[1] = ha.y; h[2] = ha.z; h[3] = ha.w;
+    h[4] = hb.x; h[5] = hb.y; h[6] = hb.z; h[7] = hb.w;
+}
+
+__global__ void __launch_bounds__(kDcThreads, 1) k_down_tc(const DownTcParams P, const __grid_constant__ CUtensorMap tmW) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t s_full[kDcStages];   // A stage landed
+    __shared__ uint64_t s_empty[kDcStages];  // the MMAs that read an A stage are done
+    __shared__ uint64_t s_done;              // the MMAs of a pass are done
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_fail;
+    __shared__ int s_pair[kDcTok];
+    __shared__ unsigned s_amax[kDcTok];  // largest |h| of each token, as fp32 bits
+    __shared__ float s_scale[kDcTok];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int slot = blockIdx.x;
+    if (slot >= *P.rw.nactive) return;
+    const int e = P.rw.active[slot];
+    const int p0 = P.rw.start[e], p1 = P.rw.start[e + 1];
+    const int m0 = blockIdx.y * kDcM;
+    if (m0 >= P.d_model) return;
+    const uint32_t sbase = (tc_smem(smem_raw) + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - tc_smem(smem_raw));
+    const uint32_t a_base = sbase;                           // kDcStages x 16 KB
+    const uint32_t b_base = sbase + kDcStages * kDcAStage;   // nst x 2 KB
+    uint8_t* b_gen = smem + kDcStages * kDcAStage;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem(&s_tmem)),
+                     "r"(kDcTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        for (int b = 0; b < kDcStages; b++) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem(&s_full[b])));
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem(&s_empty[b])));
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_smem(&s_done)));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_fail = 0;
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = s_tmem;
+    const uint32_t idesc = tc_idesc(kDcM, kDcN);
+    const int npass = (p1 - p0 + kDcTok - 1) / kDcTok;
+    const int G = npass * P.nst;                 // A stages streamed: every pass reads the whole tile
+    const int row_y = e * P.d_model + m0;        // the tile's first row in the [E d_model][d_ff] map
+    auto issue = [&](int q) {                    // A stage q into ring buffer q mod kDcStages
+        const int buf = q % kDcStages;
+        const uint32_t fb = tc_smem(&s_full[buf]);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(fb), "r"(kDcAStage) : "memory");
+        tc_tma2d(a_base + (uint32_t)buf * kDcAStage, &tmW, (q % P.nst) * kDcK, row_y, fb);
+    };
+    if (tid == 0)
+        for (int q = 0; q < min(kDcStages, G); q++) issue(q);
+
+    const int nch = P.d_ff / 8;     // 16-byte chunks of h (8 fp16) per B row inside d_ff
+    const int nchp = P.nst * 8;     // ... padded to whole stages
+    for (int pass = 0; pass < npass; pass++) {
+        const int pq = p0 + pass * kDcTok, nt = min(kDcTok, p1 - pq);
+        if (tid < kDcTok) {
+            s_pair[tid] = tid < nt ? P.rw.pairs[pq + tid] : -1;
+            s_amax[tid] = 0u;
+        }
+        __syncthreads();
+        // the largest |h| of each token (non-negative fp32 values order like their bits)
+        for (int i = tid; i < nt * nch; i += kDcThreads) {
+            const int u = i / nch, c = i - u * nch;
+            float h[8];
+            h8_of(P, s_pair[u], c, h);
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(h[j]));
+            atomicMax(&s_amax[u], __float_as_uint(m));
+        }
+        __syncthreads();
+        if (tid < kDcTok) {
+            const float m = __uint_as_float(s_amax[tid]);
+            // 2^(exponent of m - 14), kept inside [2^-100, 2^113] so that its reciprocal is finite
+            s_scale[tid] = m > 0.0f && m <= 3.0e38f ? ldexpf(1.0f, max(ilogbf(m) - 14, -100)) : 1.0f;
+        }
+        __syncthreads();
+        // B, both parts of every token (zeros for absent tokens and past d_ff), in the
+        // 128-byte swizzle: 16-byte chunk ch of row r sits at chunk ch ^ (r mod 8)
+        for (int i = tid; i < kDcTok * nchp; i += kDcThreads) {
+            const int u = i / nchp, c = i - u * nchp;
+            uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
+            if (u < nt && c < nch) {
+                float h[8];
+                h8_of(P, s_pair[u], c, h);
+                const float inv = 1.0f / s_scale[u];  // a power of two: exact
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const float v0 = h[2 * j] * inv, v1 = h[2 * j + 1] * inv;
+                    const __half a0 = __float2half_rn(v0), a1 = __float2half_rn(v1);
+                    const __half b0 = __float2half_rn(v0 - __half2float(a0)), b1 = __float2half_rn(v1 - __half2float(a1));
+                    hw[j] = (uint32_t)__half_as_ushort(a0) | ((uint32_t)__half_as_ushort(a1) << 16);
+                    lw[j] = (uint32_t)__half_as_ushort(b0) | ((uint32_t)__half_as_ushort(b1) << 16);
+                }
+                hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            const int st = c >> 3, ch = c & 7;
+            uint8_t* stage = b_gen + (size_t)st * kDcBStage;
+            *reinterpret_cast<uint4*>(stage + u * 128 + ((ch ^ u) << 4)) = hi;                // row u
+            *reinterpret_cast<uint4*>(stage + 1024 + u * 128 + ((ch ^ u) << 4)) = lo;         // row 8 + u
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // B -> the tensor core's reads
+        __syncthreads();
+        if (tid == 0) {
+            bool ok = true;
+            for (int s = 0; s < P.nst; s++) {
+                const int g = pass * P.nst + s, buf = g % kDcStages;
+                if (!tc_wait(tc_smem(&s_full[buf]), (uint32_t)(g / kDcStages) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t a_s = a_base + (uint32_t)buf * kDcAStage, b_s = b_base + (uint32_t)s * kDcBStage;
+#pragma unroll
+                for (int kk = 0; kk < kDcK / 16; kk++) {
+                    const uint64_t ad = tc_desc_sw128(a_s + 32u * kk), bd = tc_desc_sw128(b_s + 32u * kk);
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+                        "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+                        : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 tc_smem(&s_empty[buf]))
+                             : "memory");
+                // refill the buffer of the stage before this one, whose MMAs were issued first
+                const int q = g - 1 + kDcStages;
+                if (g >= 1 && q < G) {
+                    const int qb = (g - 1) % kDcStages;
+                    if (!tc_wait(tc_smem(&s_empty[qb]), (uint32_t)((g - 1) / kDcStages) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    issue(q);
+                }
+            }
+            if (!ok) s_fail = 1;
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             tc_smem(&s_done))
+                         : "memory");
+        }
+        if (!tc_wait(tc_smem(&s_done), (uint32_t)pass & 1u)) s_fail = 1;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(tmem + ((uint32_t)(32 * warp) << 16)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        const int row = m0 + 32 * warp + lane;
+        if (row < P.d_model && !s_fail) {
+#pragma unroll
+            for (int u = 0; u < kDcTok; u++)
+                if (u < nt)
+                    P.ydown[(size_t)s_pair[u] * P.d_model + row] =
+                        (__uint_as_float(v[u]) + __uint_as_float(v[kDcTok + u])) * s_scale[u];
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();  // B, the accumulator and s_pair are reused by the next pass
+        if (s_fail) break;
+    }
+    if (s_fail && tid == 0 && P.status) atomicOr(P.status, BITSMOE_ST_TIMEOUT);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kDcTmemCols) : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 // Largest dynamic shared memory k_down_t1 has been granted on each device, so that
@@ -475,19 +694,41 @@ BITSMOE_API int bitsmoe_ffn_down(const bitsmoe_ffn_dims* dims, const uint16_t* w
     FfnWS w = ffn_ws(dims, T, (uint8_t*)workspace);
     int rc = launch_route_ids(topk_ids, T * K, E, w.route, status, s);
     if (rc) return rc;
-    DownMtParams P{};
-    P.w = w_down;
-    P.yg = Y_gate;
-    P.yu = Y_up;
-    P.rw = w.route;
-    P.ydown = w.ydown;
-    P.E = E;
-    P.d_model = d_model;
-    P.d_ff = d_ff;
     const int slots = (int)std::min<int64_t>((int64_t)E, (int64_t)T * K);
-    const int rows_cta = kDmRows * (d_ff <= kDmCols ? kDmBatches : 1);
-    dim3 grid((unsigned)slots, (unsigned)((d_model + rows_cta - 1) / rows_cta));
-    k_down_mt<<<grid, kDmThreads, 0, s>>>(P);
+    if (d_ff <= kDcMaxDff && (int64_t)E * d_model < (1ll << 31)) {
+        // the tensor cores: a CTA per (expert, 128 rows)
+        CUtensorMap tmW;
+        rc = tc_tensor_map(&tmW, w_down, d_ff, E * d_model, kDcM);
+        if (rc) return rc;
+        DownTcParams P{};
+        P.yg = Y_gate;
+        P.yu = Y_up;
+        P.rw = w.route;
+        P.ydown = w.ydown;
+        P.status = status;
+        P.E = E;
+        P.d_model = d_model;
+        P.d_ff = d_ff;
+        P.nst = (d_ff + kDcK - 1) / kDcK;
+        const size_t smem = 1024 + (size_t)kDcStages * kDcAStage + (size_t)P.nst * kDcBStage;
+        cudaError_t e = cudaFuncSetAttribute(k_down_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return set_cuda_error(e);
+        dim3 grid((unsigned)slots, (unsigned)((d_model + kDcM - 1) / kDcM));
+        k_down_tc<<<grid, kDcThreads, smem, s>>>(P, tmW);
+    } else {
+        DownMtParams P{};
+        P.w = w_down;
+        P.yg = Y_gate;
+        P.yu = Y_up;
+        P.rw = w.route;
+        P.ydown = w.ydown;
+        P.E = E;
+        P.d_model = d_model;
+        P.d_ff = d_ff;
+        const int rows_cta = kDmRows * (d_ff <= kDmCols ? kDmBatches : 1);
+        dim3 grid((unsigned)slots, (unsigned)((d_model + rows_cta - 1) / rows_cta));
+        k_down_mt<<<grid, kDmThreads, 0, s>>>(P);
+    }
     rc = check_launch();
     if (rc) return rc;
     return launch_combine(topk_ids, gate_w, w.ydown, out, T, K, E, d_model, s);

@@ -21,6 +21,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace bitsmoe {
 
@@ -30,7 +31,6 @@ constexpr int kTcK = 64;              // K per stage (4 MMAs of K = 16)
 constexpr int kTcCluster = 8;         // K slices per tile
 constexpr int kTcMaxStages = 4;       // stages resident at once
 constexpr int kTcBulkCols = 32;       // token tiles up to this width reduce by bulk copies (measured: faster at 16, slower at 64)
-constexpr long long kTcWaitNs = 2000000000LL;
 
 struct TcParams {
     const uint16_t* phi_t;
@@ -44,49 +44,6 @@ struct TcParams {
     uint32_t stage_bytes;
     uint32_t recv_off;  // byte offset of the receive slices (bulk reduction)
 };
-
-__device__ __forceinline__ uint32_t tc_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzled
-// layout that a TMA tile of 64 fp16 K-elements per row writes: start address,
-// leading byte offset (unused for this layout; 16 B), stride byte offset between
-// 8-row groups (1024 B), descriptor version 1, layout type 2 (128-byte swizzle).
-// A K step of 16 elements inside the 128-byte row advances the start by 32 B.
-__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024u >> 4) << 32) | (1ull << 46) |
-           (2ull << 61);
-}
-
-// Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, both K-major.
-__host__ __device__ constexpr uint32_t tc_idesc(int m, int n) {
-    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-
-// 2-D TMA tile load (no multicast) into shared memory, completing on an mbarrier.
-__device__ __forceinline__ void tc_tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
-    long long t0;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-    for (;;) {
-        uint32_t ok;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        long long t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        if (t - t0 > kTcWaitNs) return false;
-    }
-}
 
 __global__ void __launch_bounds__(kTcThreads, 1) k_proj_tc(const TcParams P, const __grid_constant__ CUtensorMap tmA,
                                                            const __grid_constant__ CUtensorMap tmB) {
@@ -287,7 +244,7 @@ bool proj_tc_supported(int T, int d_in, int r) {
 
 // A 2-D fp16 tensor map over rows x d_in (row-major), boxes of 64 K-elements x
 // box_rows rows in the 128-byte swizzle; rows past the end read as zeros.
-static int tc_tensor_map(CUtensorMap* map, const uint16_t* base, int d_in, int rows, int box_rows) {
+int tc_tensor_map(CUtensorMap* map, const uint16_t* base, int d_in, int rows, int box_rows) {
     const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
     const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)box_rows};

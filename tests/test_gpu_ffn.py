@@ -24,18 +24,19 @@ SHAPES = [
     ("ragged", 37, 24, 6, 3, (1, 5), "softmax_topk"),
     ("min_dff", 40, 8, 3, 2, (1, 3), "softmax_topk"),
     ("wide_t1", 96, 8192, 8, 8, (1, 2), "softmax_topk"),   # top_k x d_ff too big for one CTA: grouped path at T = 1
+    ("crowded", 256, 64, 4, 2, (48,), "softmax_topk"),     # ~24 tokens per expert: several tensor-core passes
     ("qwen", 2048, 768, 128, 8, (1, 8, 64), "uniform"),
     ("mixtral", 4096, 14336, 8, 2, (1, 16), "zipf"),
 ]
 
 
-def _inputs(name, d_model, d_ff, E, K, T, routing, seed, g_scale=2.0):
+def _inputs(name, d_model, d_ff, E, K, T, routing, seed, g_scale=2.0, u_scale=1.0):
     cfg = synth.LayerConfig(name, d_model, d_ff, E, K, min(d_model, 64), T, ((1, 1.0),), routing=routing, seed=seed)
     dev = torch.device("cuda")
     gen = synth.make_generator(seed, dev)
     w = synth.make_down(cfg, gen, dev)
     yg = (torch.randn((T, K, d_ff), generator=gen, device=dev) * g_scale).contiguous()
-    yu = torch.randn((T, K, d_ff), generator=gen, device=dev).contiguous()
+    yu = (torch.randn((T, K, d_ff), generator=gen, device=dev) * u_scale).contiguous()
     ids, gw = synth.make_routing(cfg, gen, dev, T)
     return w, yg, yu, ids, gw
 
@@ -96,6 +97,18 @@ def test_ffn_down_launch_counts():
 def test_ffn_down_saturated_silu(T, orc):
     """|gate| up to ~100: SiLU saturates to v and to 0 (e^-v overflows to Inf)."""
     w, yg, yu, ids, gw = _inputs("sat", 64, 64, 4, 2, T, "softmax_topk", seed=950 + T, g_scale=30.0)
+    out, st = _run(w, yg, yu, ids, gw)
+    assert st == 0 and torch.isfinite(out).all()
+    ref, _ = _oracle(orc, w, yg, yu, ids, gw)
+    assert rel_err(out.cpu().numpy(), ref) <= TOL
+
+
+@pytest.mark.parametrize("T", [1, 6])
+def test_ffn_down_beyond_fp16_range(T, orc):
+    """|h| up to ~1e7 (far past fp16's 65504): the grouped tensor-core kernel scales each
+    token's h by a power of two before splitting it into fp16 parts."""
+    w, yg, yu, ids, gw = _inputs("big", 128, 256, 4, 2, T, "softmax_topk", seed=955 + T, g_scale=3000.0,
+                                 u_scale=1000.0)
     out, st = _run(w, yg, yu, ids, gw)
     assert st == 0 and torch.isfinite(out).all()
     ref, _ = _oracle(orc, w, yg, yu, ids, gw)
