@@ -49,6 +49,9 @@ def parse():
                          "fp16 down projection), with the down kernel's own roofline")
     ap.add_argument("--ffn-two-calls", action="store_true",
                     help="with --ffn: run each step as bitsmoe_layer_forward then bitsmoe_ffn_down")
+    ap.add_argument("--ssd", action="store_true",
+                    help="time the offline step instead: the shared-basis decomposition of one projection's experts, "
+                         "widths by descending amplitude, quantisation and packing")
     ap.add_argument("--clock-window", type=float, default=0.25,
                     help="seconds of untimed replays of the same loop before the timed steps, during which (and "
                          "during the timed steps) the SM clock is sampled")
@@ -797,6 +800,87 @@ def run_ffn(args, dist):
         print(json.dumps(line), flush=True)
 
 
+def fp32_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """fp32 FMA throughput from the unit counts: 128 lanes per SM, 2 flops per FMA."""
+    return 128 * 2 * sms * sm_mhz * 1e6 / 1e12
+
+
+def run_ssd(args, dist):
+    """The offline step for one projection of the configuration's shape, as
+    layer.decompose_and_pack runs it: the shared-basis decomposition of seeded
+    synthetic expert matrices W_e ~ N(0, 1/d_in) (fp32), the widths of the
+    configuration's allocation by descending amplitude (host), quantisation and
+    packing.  Each repetition is timed with CUDA events per stage."""
+    import torch
+    from mixed_precision_decode_b200 import bitsmoe as B
+    from mixed_precision_decode_b200 import synth
+    from mixed_precision_decode_b200.layer import PackedProjection
+
+    cfg = synth.CONFIGS[args.config]
+    E, d_out, d_in, r = cfg.n_experts, cfg.d_out, cfg.d_in, cfg.rank
+    dev = torch.device("cuda")
+    gen = synth.make_generator(30_000 + 1000 * dist.rank, dev)
+    W = (torch.randn((E, d_out, d_in), generator=gen, device=dev) * d_in ** -0.5).contiguous()
+    counts = synth.width_counts(cfg)
+    order, cnt = [b for b, _ in counts], [n for _, n in counts]
+    n_ws = B.ssd_workspace_bytes(E, d_out, d_in, r)
+    ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
+    phi_t = torch.empty((r, d_in), dtype=torch.float16, device=dev)
+    amps = torch.empty((E, r), dtype=torch.float32, device=dev)
+    comps = torch.empty((E, r, d_out), dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def once(timing):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        B.ssd_decompose(W, r, phi_t, amps, comps, ws, n_ws, status=st)
+        ev[1].record(stream)
+        torch.cuda.synchronize()  # the stages run one after another
+        t0 = time.perf_counter()
+        widths = torch.from_numpy(B.assign_widths(amps.cpu().numpy(), order, cnt))  # D2H of a, host sort
+        t_w = time.perf_counter() - t0
+        ev_p0 = torch.cuda.Event(enable_timing=True)
+        ev_p0.record(stream)
+        pk = PackedProjection.from_factors(phi_t, amps, comps, widths, cfg.top_k, status=st)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        if timing is not None:
+            timing["decompose"].append(ev[0].elapsed_time(ev[1]))
+            timing["widths"].append(t_w * 1e3)
+            timing["pack"].append(ev_p0.elapsed_time(ev[2]))
+        return pk
+
+    for _ in range(max(1, args.warmup)):
+        once(None)
+    timing = {"decompose": [], "widths": [], "pack": []}
+    dist.barrier()
+    for _ in range(args.steps):
+        pk = once(timing)
+    dist.barrier()
+    assert B.read_status(st) == 0
+    med = {k: sorted(v)[len(v) // 2] for k, v in timing.items()}
+    total = med["decompose"] + med["widths"] + med["pack"]
+    total_max = dist.max(total)
+    flops = 2 * 2 * (E * d_out) * d_in * r  # W_cat^T W_cat and W_cat Phi
+    peak = fp32_peak_tflops(1965.0)
+    ach = flops / (med["decompose"] * 1e-3) / 1e12
+    line = {"metric": "offline decomposition + widths + packing time per projection", "value": total_max,
+            "unit": "ms", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_max, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic expert matrices N(0, 1/d_in), seeded",
+            "config": {"workload": f"{cfg.name}: one projection, {E} experts of {d_out} x {d_in}, rank {r}",
+                       "widths": str(counts)},
+            "stages_ms": med,
+            "roofline": {"bound": "alu", "kernel": "decomposition (two fp32 GEMMs in cuBLAS, fp32 eigensolver)",
+                         "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                         "peak_kind": "fp32 FMA units x clocks.max.sm (1965 MHz)",
+                         "flops_per_step": flops, "duration_us": med["decompose"] * 1e3},
+            "blob_bytes": pk.plan.blob_bytes}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def kernels_per_step(wl) -> int:
     from mixed_precision_decode_b200 import bitsmoe as B
     L = wl.layers[0]
@@ -955,6 +1039,8 @@ def main():
             run_reference(args, dist)
         elif args.ffn:
             run_ffn(args, dist)
+        elif args.ssd:
+            run_ssd(args, dist)
         else:
             run_ours(args, dist)
     finally:

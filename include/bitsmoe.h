@@ -82,6 +82,8 @@ extern "C" {
 #define BITSMOE_ST_PLANMISMATCH 16 /* device widths disagree with the plan's widths */
 #define BITSMOE_ST_BOUNDS 32       /* bounds-checked build only: a computed index fell outside its
                                       buffer; that access was skipped (outputs of the call invalid) */
+#define BITSMOE_ST_NOCONVERGE 64   /* bitsmoe_ssd_decompose: the eigensolver did not converge (or met a
+                                      non-finite value); the outputs of the call are invalid */
 
 typedef struct {
     int32_t d_in;      /* input width of the projection (rows of Phi) */
@@ -310,6 +312,45 @@ int bitsmoe_ffn_launches(const bitsmoe_plan *gate, const bitsmoe_plan *up, int32
 int bitsmoe_ffn_forward(const bitsmoe_proj_io *gate, const bitsmoe_proj_io *up, const uint16_t *w_down,
                         const uint16_t *X, const int32_t *topk_ids, const float *gate_w, int32_t T, float *out,
                         void *workspace, uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* ---- the offline step before the decode path: decomposition and widths ----
+ * Shared-basis spectral decomposition of one projection's experts (study-note page,
+ * Methodology: first split, W_cat = U S Phi^T over the experts stacked vertically,
+ * (E d_out) x d_in, Phi the shared input basis, P = U S = W_cat Phi; second split,
+ * a_{e,k} = ||P_e[:,k]||, p_{e,k} = P_e[:,k] / a_{e,k}, so that
+ * W_e = sum_k a_{e,k} p_{e,k} phi_k^T).  The right singular vectors and the
+ * singular values are taken as the eigenvectors and the square roots of the
+ * eigenvalues of the Gram matrix W_cat^T W_cat (fp32 GEMMs in cuBLAS without TF32,
+ * the fp32 symmetric eigensolver of cuSOLVER; both loaded on first use); the r
+ * largest are kept, in descending order, each phi_k with the sign that makes its
+ * entry of largest magnitude positive.  The outputs are the inputs of
+ * bitsmoe_compute_scales / bitsmoe_pack and of the decode path.  Needs a GPU. */
+
+/* Workspace bytes of bitsmoe_ssd_decompose (0 for bad dims, or when cuBLAS or
+ * cuSOLVER cannot be loaded or no device is usable). */
+uint64_t bitsmoe_ssd_workspace_bytes(int32_t n_experts, int32_t d_out, int32_t d_in, int32_t rank);
+
+/*   W dev [E][d_out][d_in] f32 (the expert matrices), 1 <= rank <= d_in;
+ *   phi_t dev [rank][d_in] fp16 (out: row k = phi_k), phi_t32 dev [rank][d_in] f32
+ *   (out: the same in fp32) or NULL, sigma dev [rank] f32 (out: the singular
+ *   values) or NULL, amps dev [E][rank] f32 (out), comps dev
+ *   [E][rank][d_out] f32 (out: unit p_{e,k}; 0 where a = 0), workspace dev
+ *   (>= bitsmoe_ssd_workspace_bytes, 256-byte aligned), status dev or NULL
+ *   (BITSMOE_ST_NOCONVERGE).  Errors: EINVAL, ESIZE, ECUDA (also when cuBLAS or
+ *   cuSOLVER cannot be loaded). */
+int bitsmoe_ssd_decompose(const float *W, int32_t n_experts, int32_t d_out, int32_t d_in, int32_t rank,
+                          uint16_t *phi_t, float *phi_t32, float *sigma, float *amps, float *comps, void *workspace,
+                          uint64_t workspace_bytes, int32_t *status, void *stream);
+
+/* Widths by descending amplitude within each expert, ties to the lower k (the
+ * study-note page, Usage, gives the width set; this call takes the allocation's
+ * counts): per expert the counts[0] components of largest a get
+ * widths_in_order[0], the next counts[1] get widths_in_order[1], and so on.
+ *   amps_host [E][r] f32, widths_in_order [n] in {0,1,2,3,4,6,8,16}, counts [n]
+ *   summing to r, widths_host [E][r] u8 (out).  Host only.
+ * Errors: EINVAL (NULL, counts that do not sum to r), EWIDTH. */
+int bitsmoe_assign_widths(const float *amps_host, int32_t n_experts, int32_t rank, const uint8_t *widths_in_order,
+                          const int32_t *counts, int32_t n, uint8_t *widths_host);
 
 /* Waits for `stream`, then copies the device status word to *out_host.
  * Errors: EINVAL, ECUDA. */

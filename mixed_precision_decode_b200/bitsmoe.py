@@ -20,6 +20,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
 
 OK, EINVAL, EWIDTH, ESIZE, ECUDA, EFORMAT, ENOMEM = 0, -1, -2, -3, -4, -5, -6
 ST_NONFINITE, ST_BADSCALE, ST_BADEXPERT, ST_TIMEOUT, ST_PLANMISMATCH, ST_BOUNDS = 1, 2, 4, 8, 16, 32
+ST_NOCONVERGE = 64
 
 # Every symbol include/bitsmoe.h declares.
 EXPORTS = (
@@ -29,7 +30,8 @@ EXPORTS = (
     "bitsmoe_expert_forward", "bitsmoe_layer_workspace_bytes", "bitsmoe_layer_launches", "bitsmoe_layer_forward",
     "bitsmoe_layer_forward_chained", "bitsmoe_layer_forward_t1_noalloc", "bitsmoe_ffn_down_workspace_bytes",
     "bitsmoe_ffn_down_launches", "bitsmoe_ffn_down", "bitsmoe_ffn_workspace_bytes", "bitsmoe_ffn_launches",
-    "bitsmoe_ffn_forward", "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
+    "bitsmoe_ffn_forward", "bitsmoe_ssd_workspace_bytes", "bitsmoe_ssd_decompose", "bitsmoe_assign_widths",
+    "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
 )
 
 
@@ -96,6 +98,9 @@ def lib() -> ctypes.CDLL:
             "bitsmoe_ffn_launches": ([vp, vp, i32], ctypes.c_int),
             "bitsmoe_ffn_forward": ([ctypes.POINTER(ProjIO), ctypes.POINTER(ProjIO), vp, vp, vp, vp, i32, vp, vp, u64,
                                      vp, vp], ctypes.c_int),
+            "bitsmoe_ssd_workspace_bytes": ([i32, i32, i32, i32], u64),
+            "bitsmoe_ssd_decompose": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, u64, vp, vp], ctypes.c_int),
+            "bitsmoe_assign_widths": ([vp, i32, i32, vp, vp, i32, vp], ctypes.c_int),
             "bitsmoe_read_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "bitsmoe_strerror": ([ctypes.c_int], ctypes.c_char_p),
             "bitsmoe_version": ([], ctypes.c_int),
@@ -291,6 +296,32 @@ def ffn_forward(gate: ProjIO, up: ProjIO, w_down, X, topk_ids, gate_w, T: int, o
     _check(lib().bitsmoe_ffn_forward(ctypes.byref(gate), ctypes.byref(up), _ptr(w_down), _ptr(X), _ptr(topk_ids),
                                      _ptr(gate_w), T, _ptr(out), _ptr(workspace), workspace_bytes, _ptr(status),
                                      _stream(stream)), "ffn_forward")
+
+
+def ssd_workspace_bytes(n_experts: int, d_out: int, d_in: int, rank: int) -> int:
+    return int(lib().bitsmoe_ssd_workspace_bytes(n_experts, d_out, d_in, rank))
+
+
+def ssd_decompose(W, rank: int, phi_t, amps, comps, workspace, workspace_bytes: int, sigma=None, phi_t32=None,
+                  status=None, stream=None):
+    """W [E][d_out][d_in] f32 (GPU) -> phi_t [rank][d_in] fp16, amps [E][rank], comps [E][rank][d_out]."""
+    E, d_out, d_in = W.shape
+    _check(lib().bitsmoe_ssd_decompose(_ptr(W), E, d_out, d_in, rank, _ptr(phi_t), _ptr(phi_t32), _ptr(sigma),
+                                       _ptr(amps), _ptr(comps), _ptr(workspace), workspace_bytes, _ptr(status),
+                                       _stream(stream)),
+           "ssd_decompose")
+
+
+def assign_widths(amps_host, widths_in_order, counts) -> np.ndarray:
+    """Widths [E][r] u8 by descending amplitude within each expert (host)."""
+    a = np.ascontiguousarray(np.asarray(amps_host, dtype=np.float32))
+    E, r = a.shape
+    wo = np.ascontiguousarray(np.asarray(widths_in_order, dtype=np.uint8))
+    ct = np.ascontiguousarray(np.asarray(counts, dtype=np.int32))
+    out = np.zeros((E, r), np.uint8)
+    _check(lib().bitsmoe_assign_widths(a.ctypes.data, E, r, wo.ctypes.data, ct.ctypes.data, len(wo), out.ctypes.data),
+           "assign_widths")
+    return out
 
 
 def read_status(status, stream=None) -> int:

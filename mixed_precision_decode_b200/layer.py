@@ -47,6 +47,32 @@ class PackedProjection:
         return tot
 
 
+def decompose_and_pack(W: torch.Tensor, rank: int, widths_in_order, counts, top_k: int, status=None,
+                       stream=None) -> tuple["PackedProjection", dict]:
+    """The offline step before the decode path, on the GPU: the shared-basis spectral
+    decomposition of one projection's expert matrices W [E][d_out][d_in] (f32),
+    widths by descending amplitude (counts[j] components of each expert at
+    widths_in_order[j]), then quantisation and packing.  Returns the packed
+    projection and the decomposition (phi_t, sigma, amps, comps, widths)."""
+    E, d_out, d_in = W.shape
+    dev = W.device
+    n = B.ssd_workspace_bytes(E, d_out, d_in, rank)
+    if n == 0:
+        raise B.BitsMoEError(B.ECUDA, "ssd_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    phi_t = torch.empty((rank, d_in), dtype=torch.float16, device=dev)
+    phi_t32 = torch.empty((rank, d_in), dtype=torch.float32, device=dev)
+    sigma = torch.empty(rank, dtype=torch.float32, device=dev)
+    amps = torch.empty((E, rank), dtype=torch.float32, device=dev)
+    comps = torch.empty((E, rank, d_out), dtype=torch.float32, device=dev)
+    B.ssd_decompose(W.contiguous(), rank, phi_t, amps, comps, ws, n, sigma=sigma, phi_t32=phi_t32, status=status,
+                    stream=stream)
+    del ws
+    widths = torch.from_numpy(B.assign_widths(amps.cpu().numpy(), widths_in_order, counts))
+    pk = PackedProjection.from_factors(phi_t, amps, comps, widths, top_k, status=status, stream=stream)
+    return pk, {"phi_t": phi_t, "phi_t32": phi_t32, "sigma": sigma, "amps": amps, "comps": comps, "widths": widths}
+
+
 class SpectralMoELayer:
     """Gate and up projections of one MoE layer in shared-spectral form."""
 

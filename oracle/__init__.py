@@ -283,6 +283,24 @@ def moe_ffn_forward(blob_gate, blob_up, phi_t_gate_bits, phi_t_up_bits, x_bits, 
     return out, lf["gate"]["status"] | lf["up"]["status"] | st
 
 
+def assign_widths(amps: np.ndarray, widths_in_order, counts) -> np.ndarray:
+    """Widths [E][r] by descending amplitude within each expert, ties to the lower k:
+    the counts[0] largest get widths_in_order[0], the next counts[1] widths_in_order[1], ...
+    (the configurations' allocation rule; the pages' allocator chooses the counts)."""
+    a = np.asarray(amps, dtype=np.float64)
+    E, r = a.shape
+    assert sum(int(c) for c in counts) == r
+    out = np.zeros((E, r), np.uint8)
+    for e in range(E):
+        order = sorted(range(r), key=lambda k: (-a[e, k], k))
+        pos = 0
+        for b, c in zip(widths_in_order, counts):
+            for k in order[pos:pos + int(c)]:
+                out[e, k] = b
+            pos += int(c)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # offline shared-basis decomposition (used by the reconstruction check)
 # ---------------------------------------------------------------------------

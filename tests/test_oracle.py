@@ -598,3 +598,24 @@ def test_ffn_routing_invariants(orc):
     assert np.allclose(out5[0], out6[0], rtol=1e-14, atol=1e-14) and np.array_equal(out5[1:], out[1:])
     out0, st0 = orc.ffn_down(Yg[:0], Yu[:0], W.view(np.uint16), ids[:0], g[:0])
     assert out0.shape == (0, d_model) and st0 == 0
+
+
+# --------------------------------------------------------------------------
+# widths by descending amplitude (the configurations' allocation rule)
+# --------------------------------------------------------------------------
+
+def test_assign_widths_brute_force(orc):
+    """Per expert: the counts per width are exact; a component never gets a width
+    listed later than one of smaller amplitude; among equal amplitudes the lower k
+    comes first.  Checked against every pair of components."""
+    rng = np.random.default_rng(81)
+    order, counts = (8, 4, 3, 2, 1, 0), (1, 2, 3, 4, 2, 2)
+    a = rng.choice([0.5, 1.0, 1.5, 2.0, 3.0], size=(3, 14)).astype(np.float32)  # many ties
+    w = orc.assign_widths(a, order, counts)
+    rank = {b: i for i, b in enumerate(order)}
+    for e in range(3):
+        assert [int((w[e] == b).sum()) for b in order] == list(counts)
+        for j in range(14):
+            for k in range(14):
+                if a[e, j] > a[e, k] or (a[e, j] == a[e, k] and j < k):
+                    assert rank[int(w[e, j])] <= rank[int(w[e, k])]
