@@ -83,10 +83,11 @@ def lib():
         L.orc_shared_proj.restype = None
         L.orc_expert_forward.argtypes = [c_u8p, ctypes.c_uint64, c_f64p, c_i32p, c_f32p, ctypes.c_int,
                                          ctypes.c_int, c_f64p, c_f64p, c_i32p]
+        L.orc_fqcm_eps.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, c_f32p, c_f64p]
         L.orc_ffn_down.argtypes = [c_f64p, c_f64p, c_u16p, c_i32p, c_f32p, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, c_f64p, c_i32p]
         for f in ("orc_compute_scales", "orc_pack", "orc_blob_parse", "orc_unpack", "orc_dequant_expert",
-                  "orc_expert_forward", "orc_ffn_down"):
+                  "orc_expert_forward", "orc_ffn_down", "orc_fqcm_eps"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -299,6 +300,85 @@ def assign_widths(amps: np.ndarray, widths_in_order, counts) -> np.ndarray:
                 out[e, k] = b
             pos += int(c)
     return out
+
+
+# ---------------------------------------------------------------------------
+# the allocation of widths: FQCM cost and the bit budget (third split, Usage)
+# ---------------------------------------------------------------------------
+WIDTH_SET = (0, 1, 2, 3, 4, 6, 8, 16)  # the order of the eps arrays
+
+
+def fqcm_eps(comps: np.ndarray) -> np.ndarray:
+    """eps [E][r][8] (fp64): squared error of storing each unit direction at each width
+    of WIDTH_SET (the pages' width-dependent distortion, read as ||p - stored p||^2)."""
+    comps = _c(comps, np.float32)
+    E, r, d_out = comps.shape
+    eps = np.zeros((E, r, 8), np.float64)
+    _check(lib().orc_fqcm_eps(E, r, d_out, _p(comps, ctypes.c_float), _p(eps, ctypes.c_double)), "fqcm_eps")
+    return eps
+
+
+def fqcm_beta(Z: np.ndarray, ids: np.ndarray, gate_w: np.ndarray, n_experts: int) -> np.ndarray:
+    """beta [E][r] (fp64): the activation importance of each spectral direction for each
+    expert over calibration tokens, sum over the (token, slot) pairs routed to e of
+    g * z_k^2, with z = Phi^T x (third split: beta = phi_k^T X_e G_e X_e^T phi_k)."""
+    Z = np.asarray(Z, np.float64)
+    ids = np.asarray(ids)
+    g = np.asarray(gate_w, np.float64)
+    T, r = Z.shape
+    beta = np.zeros((n_experts, r), np.float64)
+    for t in range(T):
+        for j in range(ids.shape[1]):
+            e = int(ids[t, j])
+            if 0 <= e < n_experts:
+                beta[e] += g[t, j] * Z[t] ** 2
+    return beta
+
+
+def allocate_widths(amps: np.ndarray, beta: np.ndarray, eps: np.ndarray, d_out: int, budget_bits: int):
+    """Widths [E][r] minimising sum L_{e,k}(b) = a^2 beta eps_b under sum d_out b <= budget_bits
+    (the pages: a bit budget, every candidate width of every component considered
+    jointly).  Solved as the linear relaxation of this multiple-choice knapsack:
+    per component, the lower convex hull of its (bits, loss) points from width 0;
+    then every hull segment of every component, in order of loss saved per bit
+    (ties: lower component, then earlier segment), taken while it fits; the first
+    that does not fit ends the allocation.  Returns (widths, total loss)."""
+    a = np.asarray(amps, np.float64)
+    beta = np.asarray(beta, np.float64)
+    eps = np.asarray(eps, np.float64)
+    E, r = a.shape
+    segs = []
+    choice = np.zeros(E * r, np.int64)  # index into WIDTH_SET
+    for c in range(E * r):
+        e, k = divmod(c, r)
+        imp = a[e, k] * a[e, k] * beta[e, k]
+        pts = [(d_out * b, imp * eps[e, k, i], i) for i, b in enumerate(WIDTH_SET)]
+        hull = [pts[0]]
+        for pt in pts[1:]:
+            if pt[1] >= hull[-1][1]:
+                continue  # more bits and no less loss
+            while len(hull) >= 2:
+                A, Bp = hull[-2], hull[-1]
+                # Bp leaves the lower hull unless the slope A->Bp is steeper than A->pt
+                if (Bp[1] - A[1]) * (pt[0] - A[0]) >= (pt[1] - A[1]) * (Bp[0] - A[0]):
+                    hull.pop()
+                else:
+                    break
+            hull.append(pt)
+        for s in range(len(hull) - 1):
+            gain = hull[s][1] - hull[s + 1][1]
+            cost = hull[s + 1][0] - hull[s][0]
+            segs.append((gain / cost, c, s, cost, hull[s + 1][2]))
+    segs.sort(key=lambda x: (-x[0], x[1], x[2]))
+    used = 0
+    for eff, c, s, cost, wi in segs:
+        if used + cost > budget_bits:
+            break
+        used += cost
+        choice[c] = wi
+    widths = np.array([WIDTH_SET[i] for i in choice], np.uint8).reshape(E, r)
+    loss = sum(a[c // r, c % r] ** 2 * beta[c // r, c % r] * eps[c // r, c % r, choice[c]] for c in range(E * r))
+    return widths, float(loss)
 
 
 # ---------------------------------------------------------------------------

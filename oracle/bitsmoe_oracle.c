@@ -632,3 +632,58 @@ int orc_ffn_down(const double *Yg, const double *Yu, const uint16_t *w_down, con
     if (status) *status |= st;
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Width-dependent distortion of each component (the FQCM cost's third factor). */
+/* ------------------------------------------------------------------------- */
+
+/* The pages name a width-dependent distortion eps_{e,k,b} but do not define it.
+ * Read here as the squared error of storing the unit direction at width b:
+ *   eps_{e,k,b} = sum_i (p_i - w_i)^2  (fp64),
+ * w the stored value: b in 1..8, the quantiser above with the component's fp16
+ * scale for that width, w = s (q - (2^b - 1)/2); b = 16, the fp16 value; b = 0,
+ * w = 0 (so eps = ||p||^2).  Widths in the order 0,1,2,3,4,6,8,16: eps is
+ * [E][r][8].  A component with a non-finite element gets NaN at every width. */
+static const int ORC_WIDTH_SET[8] = {0, 1, 2, 3, 4, 6, 8, 16};
+
+int orc_fqcm_eps(int E, int r, int d_out, const float *comps, double *eps) {
+    if (!orc_dims_ok(E, r, d_out) || !comps || !eps) return ORC_EINVAL;
+    for (int e = 0; e < E; e++)
+        for (int k = 0; k < r; k++) {
+            const float *p = comps + ((size_t)e * r + k) * (size_t)d_out;
+            double *out = eps + ((size_t)e * r + k) * 8;
+            float m = 0.0f;
+            int bad = 0;
+            for (int i = 0; i < d_out; i++) {
+                if (!isfinite(p[i])) bad = 1;
+                float a = fabsf(p[i]);
+                if (a > m) m = a;
+            }
+            for (int wi = 0; wi < 8; wi++) {
+                const int b = ORC_WIDTH_SET[wi];
+                if (bad) {
+                    out[wi] = NAN;
+                    continue;
+                }
+                uint16_t sh = 0;
+                if (b != 0 && b != 16) sh = orc_f32_to_f16((2.0f * m) / (float)((1 << b) - 1));
+                double acc = 0.0;
+                for (int i = 0; i < d_out; i++) {
+                    double w;
+                    if (b == 0) {
+                        w = 0.0;
+                    } else if (b == 16) {
+                        w = orc_f16_to_f64(orc_f32_to_f16(p[i]));
+                    } else {
+                        int32_t st = 0;
+                        uint32_t q = orc_quantise(p[i], b, sh, &st);
+                        w = orc_dequant(b, (uint16_t)q, sh);
+                    }
+                    const double d = (double)p[i] - w;
+                    acc += d * d;
+                }
+                out[wi] = acc;
+            }
+        }
+    return ORC_OK;
+}

@@ -619,3 +619,110 @@ def test_assign_widths_brute_force(orc):
             for k in range(14):
                 if a[e, j] > a[e, k] or (a[e, j] == a[e, k] and j < k):
                     assert rank[int(w[e, j])] <= rank[int(w[e, k])]
+
+
+# --------------------------------------------------------------------------
+# FQCM: distortion per width, activation importance, the bit-budget allocation
+# --------------------------------------------------------------------------
+
+def test_fqcm_eps_closed_forms(orc):
+    """p = (1.5, -1.5, 0.5, -0.5): at 2 bits the scale is fp16(3 / 3) = 1 and the levels
+    are +-0.5, +-1.5, so eps = 0; at 1 bit the levels are +-1.5 (scale 3) and the two
+    small entries land on the far levels, eps = 1 + 1 = 2; at 0 bits eps = ||p||^2 = 5;
+    every entry is an fp16 value, so eps(16) = 0.  p = (1.5, 0.2, 0, 0) at 2 bits: 0.2 and
+    both zeros go to level 0.5 (the mid-rise levels have no 0), eps = 0.3^2 + 2 (0.5)^2.
+    fp16 rounding of 0.1 against numpy's float16."""
+    p = np.zeros((1, 3, 4), np.float32)
+    p[0, 0] = [1.5, -1.5, 0.5, -0.5]
+    p[0, 1] = [1.5, 0.2, 0.0, 0.0]
+    p[0, 2] = [0.1, 0.0, 0.0, 0.0]
+    eps = orc.fqcm_eps(p)
+    W = {b: i for i, b in enumerate(orc.WIDTH_SET)}
+    assert eps[0, 0, W[2]] == 0.0 and eps[0, 0, W[16]] == 0.0
+    assert eps[0, 0, W[1]] == 2.0 and eps[0, 0, W[0]] == 5.0
+    assert abs(eps[0, 1, W[2]] - ((float(np.float32(0.2)) - 0.5) ** 2 + 2 * 0.25)) <= 1e-15
+    h = float(np.float16(np.float32(0.1)))
+    assert eps[0, 2, W[16]] == (float(np.float32(0.1)) - h) ** 2
+
+
+def test_fqcm_eps_falls_with_width_on_average(orc):
+    """On random unit vectors eps falls with every width from 2 bits on.  At 1 bit the
+    mid-rise levels are +-max|p|, which overshoot most entries: on average eps(1) is
+    above eps(0) = ||p||^2 = 1 (so an allocation never prefers 1 bit to 0 there)."""
+    rng = np.random.default_rng(91)
+    p = rng.standard_normal((2, 50, 64)).astype(np.float32)
+    p /= np.linalg.norm(p, axis=2, keepdims=True)
+    m = orc.fqcm_eps(p).mean(axis=(0, 1))
+    assert abs(m[0] - 1.0) <= 1e-6 and m[1] > m[0] and np.all(np.diff(m[1:]) < 0)
+
+
+def test_fqcm_beta_closed_form_and_H_route(orc):
+    """beta[e][k] = sum over pairs routed to e of g z_k^2 (a closed form on a 2 x 2 case),
+    and equal to diag(Phi^T H_e Phi) with H_e = sum g x x^T built by numpy matmuls."""
+    Z = np.array([[1.0, 2.0], [3.0, 0.0]])
+    ids = np.array([[0, 1], [1, 0]])
+    g = np.array([[0.5, 0.25], [1.0, 2.0]])
+    beta = orc.fqcm_beta(Z, ids, g, 2)
+    assert np.array_equal(beta, np.array([[18.5, 2.0], [9.25, 1.0]]))
+    rng = np.random.default_rng(92)
+    T, d_in, r, E, K = 6, 10, 7, 3, 2
+    X = rng.standard_normal((T, d_in))
+    Phi, _ = np.linalg.qr(rng.standard_normal((d_in, r)))
+    ids = rng.integers(0, E, (T, K))
+    g = rng.uniform(0, 1, (T, K))
+    beta = orc.fqcm_beta(X @ Phi, ids, g, E)
+    for e in range(E):
+        H = sum(g[t, j] * np.outer(X[t], X[t]) for t in range(T) for j in range(K) if ids[t, j] == e)
+        H = H if not np.isscalar(H) else np.zeros((d_in, d_in))
+        assert np.allclose(beta[e], np.diag(Phi.T @ H @ Phi), rtol=1e-12, atol=1e-12)
+
+
+def _brute(a, beta, eps, d_out, budget, WS):
+    import itertools
+    E, r = a.shape
+    best = None
+    for combo in itertools.product(range(8), repeat=E * r):
+        bits = sum(d_out * WS[i] for i in combo)
+        if bits > budget:
+            continue
+        loss = sum(a[c // r, c % r] ** 2 * beta[c // r, c % r] * eps[c // r, c % r, i] for c, i in enumerate(combo))
+        best = loss if best is None else min(best, loss)
+    return best
+
+
+def test_allocate_widths_optimal_at_relaxation_vertices(orc):
+    """Brute force over all 8^4 width choices: at every budget where the relaxation's
+    solution is integral (the cumulative bits of its first m steps) the allocation is
+    optimal; at any budget it respects the budget and more budget never costs loss."""
+    rng = np.random.default_rng(93)
+    WS = orc.WIDTH_SET
+    E, r, d_out = 1, 4, 2
+    a = rng.uniform(0.2, 2.0, (E, r))
+    beta = rng.uniform(0.1, 3.0, (E, r))
+    eps = np.sort(rng.uniform(0, 1, (E, r, 8)), axis=2)[:, :, ::-1].copy()  # falling with width
+    eps[:, :, 0] = 1.0
+    prev = None
+    vertices = 0
+    for budget in range(0, d_out * 16 * r + 1, 2):
+        w, loss = orc.allocate_widths(a, beta, eps, d_out, budget)
+        used = int(d_out * w.astype(np.int64).sum())
+        assert used <= budget
+        if prev is not None:
+            assert loss <= prev + 1e-12
+        prev = loss
+        if used == budget:  # the relaxation's solution is integral here
+            vertices += 1
+            assert abs(loss - _brute(a, beta, eps, d_out, budget, WS)) <= 1e-12
+    assert vertices >= 8
+
+
+def test_allocate_widths_edges(orc):
+    E, r, d_out = 2, 3, 4
+    a = np.ones((E, r))
+    eps = np.tile(np.linspace(1, 0, 8), (E, r, 1))
+    w, loss = orc.allocate_widths(a, np.zeros((E, r)), eps, d_out, 10 ** 6)
+    assert np.all(w == 0) and loss == 0.0  # no importance: nothing is worth a bit
+    w, _ = orc.allocate_widths(a, np.ones((E, r)), eps, d_out, 0)
+    assert np.all(w == 0)
+    w, loss = orc.allocate_widths(a, np.ones((E, r)), eps, d_out, 10 ** 6)
+    assert np.all(w == 16) and loss == 0.0
