@@ -52,6 +52,10 @@ def parse():
     ap.add_argument("--ssd", action="store_true",
                     help="time the offline step instead: the shared-basis decomposition of one projection's experts, "
                          "widths by descending amplitude, quantisation and packing")
+    ap.add_argument("--fqcm", action="store_true",
+                    help="with --ssd: choose the widths by the FQCM cost under the configuration's average bits "
+                         "(calibration: --calib-tokens seeded tokens and routings) instead of its fixed fractions")
+    ap.add_argument("--calib-tokens", type=int, default=4096)
     ap.add_argument("--clock-window", type=float, default=0.25,
                     help="seconds of untimed replays of the same loop before the timed steps, during which (and "
                          "during the timed steps) the SM clock is sampled")
@@ -831,6 +835,12 @@ def run_ssd(args, dist):
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
+    if args.fqcm:
+        from mixed_precision_decode_b200.layer import fqcm_widths
+        xc = torch.randn((args.calib_tokens, d_in), generator=gen, device=dev).to(torch.float16)
+        ids_c, gw_c = synth.make_routing(cfg, gen, dev, args.calib_tokens)
+        avg_bits = sum(b * n for b, n in counts) / r
+
     def once(timing):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         ev[0].record(stream)
@@ -838,7 +848,10 @@ def run_ssd(args, dist):
         ev[1].record(stream)
         torch.cuda.synchronize()  # the stages run one after another
         t0 = time.perf_counter()
-        widths = torch.from_numpy(B.assign_widths(amps.cpu().numpy(), order, cnt))  # D2H of a, host sort
+        if args.fqcm:  # z of the calibration tokens on the GPU, then beta, eps and the allocation on the host
+            widths, _, _ = fqcm_widths({"phi_t": phi_t, "amps": amps, "comps": comps}, xc, ids_c, gw_c, avg_bits)
+        else:
+            widths = torch.from_numpy(B.assign_widths(amps.cpu().numpy(), order, cnt))  # D2H of a, host sort
         t_w = time.perf_counter() - t0
         ev_p0 = torch.cuda.Event(enable_timing=True)
         ev_p0.record(stream)
@@ -870,7 +883,8 @@ def run_ssd(args, dist):
             "ms_per_step": total_max, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic expert matrices N(0, 1/d_in), seeded",
             "config": {"workload": f"{cfg.name}: one projection, {E} experts of {d_out} x {d_in}, rank {r}",
-                       "widths": str(counts)},
+                       "widths": (f"FQCM allocation at {sum(b * n for b, n in counts) / r:.4f} average bits, "
+                                  f"{args.calib_tokens} seeded calibration tokens") if args.fqcm else str(counts)},
             "stages_ms": med,
             "roofline": {"bound": "alu", "kernel": "decomposition (two fp32 GEMMs in cuBLAS, fp32 eigensolver)",
                          "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,

@@ -352,6 +352,40 @@ int bitsmoe_ssd_decompose(const float *W, int32_t n_experts, int32_t d_out, int3
 int bitsmoe_assign_widths(const float *amps_host, int32_t n_experts, int32_t rank, const uint8_t *widths_in_order,
                           const int32_t *counts, int32_t n, uint8_t *widths_host);
 
+/* ---- the allocation of widths (offline, host) ----
+ * The study-note page, Methodology, third split: activation-dependent importance
+ * beta_{e,k} = sum over calibration (token, slot) pairs routed to e of
+ * g (phi_k^T x)^2, importance a_{e,k}^2 beta_{e,k}, cost L_{e,k}(b) =
+ * a^2 beta eps_{e,k,b}; Usage: widths in {0,1,2,3,4,6,8,16} chosen jointly under a
+ * bit budget (a component of d_out elements costs d_out b bits).  The pages leave
+ * eps undefined: eps_{e,k,b} = ||p_{e,k} - stored p_{e,k}||^2 at width b with this
+ * library's quantiser (0 bits: ||p||^2; 16 bits: fp16(p)).  All host, fp64, in a
+ * fixed order (results independent of the thread count).  Width index order of
+ * eps arrays: 0,1,2,3,4,6,8,16. */
+
+/* comps_host [E][r][d_out] f32 -> eps_host [E][r][8] f64 (NaN at
+ * every width for a component with a non-finite element).  Errors: EINVAL. */
+int bitsmoe_fqcm_eps(const float *comps_host, int32_t n_experts, int32_t rank, int32_t d_out, double *eps_host);
+
+/* beta_host [E][r] f64 from Z_host [T][r] f32 (z = Phi^T x of T calibration tokens,
+ * e.g. from bitsmoe_shared_proj), topk_ids_host [T][top_k], gate_w_host [T][top_k];
+ * ids outside [0, E) are skipped.  Errors: EINVAL. */
+int bitsmoe_fqcm_beta(const float *Z_host, const int32_t *topk_ids_host, const float *gate_w_host, int32_t T,
+                      int32_t top_k, int32_t n_experts, int32_t rank, double *beta_host);
+
+/* widths_host [E][r] u8 minimising sum L_{e,k}(b) under sum d_out b <= budget_bits,
+ * through the linear relaxation of this multiple-choice knapsack: per component the
+ * lower convex hull of its (bits, loss) points from width 0, then all hull segments
+ * in order of loss saved per bit (ties: lower e r + k, then earlier segment), taken
+ * while they fit, the first that does not fit ending the allocation (at budgets
+ * where the relaxation is integral this is the integer optimum).  A component
+ * whose cost is not finite keeps width 0.  loss_host (out, total cost) or NULL.
+ * amps_host [E][r] f32, beta_host [E][r] f64, eps_host [E][r][8] f64.
+ * Errors: EINVAL. */
+int bitsmoe_allocate_widths(const float *amps_host, const double *beta_host, const double *eps_host,
+                            int32_t n_experts, int32_t rank, int32_t d_out, uint64_t budget_bits,
+                            uint8_t *widths_host, double *loss_host);
+
 /* Waits for `stream`, then copies the device status word to *out_host.
  * Errors: EINVAL, ECUDA. */
 int bitsmoe_read_status(const int32_t *status_dev, void *stream, int32_t *out_host);

@@ -31,6 +31,7 @@ EXPORTS = (
     "bitsmoe_layer_forward_chained", "bitsmoe_layer_forward_t1_noalloc", "bitsmoe_ffn_down_workspace_bytes",
     "bitsmoe_ffn_down_launches", "bitsmoe_ffn_down", "bitsmoe_ffn_workspace_bytes", "bitsmoe_ffn_launches",
     "bitsmoe_ffn_forward", "bitsmoe_ssd_workspace_bytes", "bitsmoe_ssd_decompose", "bitsmoe_assign_widths",
+    "bitsmoe_fqcm_eps", "bitsmoe_fqcm_beta", "bitsmoe_allocate_widths",
     "bitsmoe_read_status", "bitsmoe_strerror", "bitsmoe_version",
 )
 
@@ -101,6 +102,9 @@ def lib() -> ctypes.CDLL:
             "bitsmoe_ssd_workspace_bytes": ([i32, i32, i32, i32], u64),
             "bitsmoe_ssd_decompose": ([vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, u64, vp, vp], ctypes.c_int),
             "bitsmoe_assign_widths": ([vp, i32, i32, vp, vp, i32, vp], ctypes.c_int),
+            "bitsmoe_fqcm_eps": ([vp, i32, i32, i32, vp], ctypes.c_int),
+            "bitsmoe_fqcm_beta": ([vp, vp, vp, i32, i32, i32, i32, vp], ctypes.c_int),
+            "bitsmoe_allocate_widths": ([vp, vp, vp, i32, i32, i32, u64, vp, vp], ctypes.c_int),
             "bitsmoe_read_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "bitsmoe_strerror": ([ctypes.c_int], ctypes.c_char_p),
             "bitsmoe_version": ([], ctypes.c_int),
@@ -322,6 +326,47 @@ def assign_widths(amps_host, widths_in_order, counts) -> np.ndarray:
     _check(lib().bitsmoe_assign_widths(a.ctypes.data, E, r, wo.ctypes.data, ct.ctypes.data, len(wo), out.ctypes.data),
            "assign_widths")
     return out
+
+
+WIDTH_SET = (0, 1, 2, 3, 4, 6, 8, 16)  # the width order of eps arrays
+
+
+def _host(a, dtype):
+    return np.ascontiguousarray(np.asarray(a, dtype=dtype))
+
+
+def fqcm_eps(comps_host) -> np.ndarray:
+    """eps [E][r][8] f64: squared error of each unit direction stored at each width."""
+    c = _host(comps_host, np.float32)
+    E, r, d_out = c.shape
+    out = np.zeros((E, r, 8), np.float64)
+    _check(lib().bitsmoe_fqcm_eps(c.ctypes.data, E, r, d_out, out.ctypes.data), "fqcm_eps")
+    return out
+
+
+def fqcm_beta(Z_host, topk_ids_host, gate_w_host, n_experts: int) -> np.ndarray:
+    """beta [E][r] f64 from z = Phi^T x of calibration tokens and their routing."""
+    Z = _host(Z_host, np.float32)
+    ids = _host(topk_ids_host, np.int32)
+    g = _host(gate_w_host, np.float32)
+    T, r = Z.shape
+    out = np.zeros((n_experts, r), np.float64)
+    _check(lib().bitsmoe_fqcm_beta(Z.ctypes.data, ids.ctypes.data, g.ctypes.data, T, ids.shape[1], n_experts, r,
+                                   out.ctypes.data), "fqcm_beta")
+    return out
+
+
+def allocate_widths(amps_host, beta_host, eps_host, d_out: int, budget_bits: int) -> tuple[np.ndarray, float]:
+    """(widths [E][r] u8, total cost) under sum d_out b <= budget_bits."""
+    a = _host(amps_host, np.float32)
+    b = _host(beta_host, np.float64)
+    e = _host(eps_host, np.float64)
+    E, r = a.shape
+    w = np.zeros((E, r), np.uint8)
+    loss = ctypes.c_double(0.0)
+    _check(lib().bitsmoe_allocate_widths(a.ctypes.data, b.ctypes.data, e.ctypes.data, E, r, d_out, int(budget_bits),
+                                         w.ctypes.data, ctypes.byref(loss)), "allocate_widths")
+    return w, float(loss.value)
 
 
 def read_status(status, stream=None) -> int:

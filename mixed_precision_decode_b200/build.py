@@ -20,7 +20,7 @@ LIB_CHECKED = os.path.join(PKG, "libbitsmoe_checked.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # No fast-math: the packer's divide and add must be IEEE round-to-nearest.
-FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE,
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden,-ffp-contract=off", "-I", INCLUDE,
          "-Xptxas", "-warn-spills"]
 
 

@@ -73,6 +73,27 @@ def decompose_and_pack(W: torch.Tensor, rank: int, widths_in_order, counts, top_
     return pk, {"phi_t": phi_t, "phi_t32": phi_t32, "sigma": sigma, "amps": amps, "comps": comps, "widths": widths}
 
 
+def fqcm_widths(dec: dict, x_calib: torch.Tensor, ids_calib: torch.Tensor, gw_calib: torch.Tensor,
+                avg_bits: float, stream=None) -> tuple[torch.Tensor, float, dict]:
+    """Widths of one decomposed projection (decompose_and_pack's second result) by the
+    FQCM cost under a budget of avg_bits per element: z = Phi^T x of the calibration
+    tokens x_calib [T][d_in] fp16 on the GPU, then on the host the activation
+    importance beta from z and the routing (ids_calib, gw_calib [T][top_k]), the
+    distortion of every component at every width, and the allocation.
+    Returns (widths [E][r] u8, total cost, {"beta", "eps"})."""
+    phi_t = dec["phi_t"]
+    r, d_in = phi_t.shape
+    E, _, d_out = dec["comps"].shape
+    T = x_calib.shape[0]
+    Z = torch.empty((T, r), dtype=torch.float32, device=phi_t.device)
+    B.shared_proj(phi_t, x_calib.contiguous(), Z, T, d_in, r, stream)
+    beta = B.fqcm_beta(Z.cpu().numpy(), ids_calib.cpu().numpy(), gw_calib.cpu().numpy(), E)
+    eps = B.fqcm_eps(dec["comps"].cpu().numpy())
+    budget = int(avg_bits * E * r * d_out)
+    widths, loss = B.allocate_widths(dec["amps"].cpu().numpy(), beta, eps, d_out, budget)
+    return torch.from_numpy(widths), loss, {"beta": beta, "eps": eps}
+
+
 class SpectralMoELayer:
     """Gate and up projections of one MoE layer in shared-spectral form."""
 

@@ -342,7 +342,8 @@ def allocate_widths(amps: np.ndarray, beta: np.ndarray, eps: np.ndarray, d_out: 
     per component, the lower convex hull of its (bits, loss) points from width 0;
     then every hull segment of every component, in order of loss saved per bit
     (ties: lower component, then earlier segment), taken while it fits; the first
-    that does not fit ends the allocation.  Returns (widths, total loss)."""
+    that does not fit ends the allocation.  A component whose cost is not finite
+    at some width keeps width 0.  Returns (widths, total loss)."""
     a = np.asarray(amps, np.float64)
     beta = np.asarray(beta, np.float64)
     eps = np.asarray(eps, np.float64)
@@ -353,6 +354,8 @@ def allocate_widths(amps: np.ndarray, beta: np.ndarray, eps: np.ndarray, d_out: 
         e, k = divmod(c, r)
         imp = a[e, k] * a[e, k] * beta[e, k]
         pts = [(d_out * b, imp * eps[e, k, i], i) for i, b in enumerate(WIDTH_SET)]
+        if not all(np.isfinite(pt[1]) for pt in pts):
+            continue  # a component without a finite cost keeps width 0
         hull = [pts[0]]
         for pt in pts[1:]:
             if pt[1] >= hull[-1][1]:

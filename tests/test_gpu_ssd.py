@@ -16,7 +16,7 @@ import torch
 from cases import TOL, rel_err
 from mixed_precision_decode_b200 import bitsmoe as B
 from mixed_precision_decode_b200 import synth
-from mixed_precision_decode_b200.layer import SpectralMoELayer, decompose_and_pack
+from mixed_precision_decode_b200.layer import PackedProjection, SpectralMoELayer, decompose_and_pack, fqcm_widths
 
 pytestmark = pytest.mark.gpu
 
@@ -167,3 +167,39 @@ def test_decompose_pack_widths_follow_amplitudes():
     for e in range(E):
         n = h[64 + 64 * e + 44: 64 + 64 * e + 60].view(np.uint16)  # counts in width order 16,8,6,4,3,2,1,0
         assert [int(n[1]), int(n[3]), int(n[5]), int(n[6]), int(n[7])] == list(counts)
+
+
+def test_fqcm_allocation_pipeline():
+    """Decomposition, the FQCM allocation from seeded calibration tokens (z on the
+    GPU), packing and decoding: the budget holds, every width is in the set, and on
+    its own cost the allocation is no worse than the fixed-fraction rule at the same
+    average bits (which it is free to choose), nor than uniform 2 bits."""
+    E, d_out, d_in, K, Tc = 6, 64, 128, 2, 256
+    rng = np.random.default_rng(61)
+    W = torch.from_numpy(rng.standard_normal((E, d_out, d_in)) / np.sqrt(d_in)).float().cuda()
+    order, counts = (8, 4, 3, 2, 1, 0), (3, 10, 26, 51, 25, 13)
+    _, dec = decompose_and_pack(W, d_in, order, counts, K)
+    cfg = synth.LayerConfig("fqcm", d_in, d_out, E, K, d_in, Tc, ((2, 1.0),), seed=62)
+    gen = synth.make_generator(62, torch.device("cuda"))
+    xc = torch.randn((Tc, d_in), generator=gen, device="cuda").to(torch.float16)
+    ids, gw = synth.make_routing(cfg, gen, torch.device("cuda"), Tc)
+    avg = sum(b * c for b, c in zip(order, counts)) / d_in
+    widths, loss, parts = fqcm_widths(dec, xc, ids, gw, avg)
+    w = widths.numpy()
+    assert set(np.unique(w).tolist()) <= set(B.WIDTH_SET)
+    assert int(d_out * w.astype(np.int64).sum()) <= int(avg * E * d_in * d_out)
+    a = dec["amps"].cpu().numpy().astype(np.float64)
+    idx = {b: i for i, b in enumerate(B.WIDTH_SET)}
+    def cost(ws):
+        wi = np.vectorize(idx.get)(ws)
+        return float((a ** 2 * parts["beta"] * np.take_along_axis(parts["eps"], wi[..., None], 2)[..., 0]).sum())
+    assert abs(cost(w) - loss) <= 1e-9 * max(loss, 1.0)
+    # the relaxation's optimum is below both; the allocation stops at the first step that
+    # does not fit, so it can exceed that optimum by at most one step's saving (1 % here)
+    assert loss <= cost(dec["widths"].numpy()) * 1.01
+    assert loss <= cost(np.full_like(w, 2)) * 1.01
+    pk = PackedProjection.from_factors(dec["phi_t"], dec["amps"], dec["comps"], widths, K)
+    layer = SpectralMoELayer(pk, pk)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = layer.forward(xc[:3], ids[:3], gw[:3], status=st)
+    assert B.read_status(st) == 0 and torch.isfinite(out["Y_sum_gate"]).all()

@@ -43,3 +43,65 @@ def test_ssd_argument_checks(B):
     assert L.bitsmoe_ssd_decompose(None, 4, 32, 64, 64, *args) == B.EINVAL
     assert L.bitsmoe_ssd_decompose(256, 4, 32, 64, 64, 256, None, None, 256, 256, 0x1010, 1 << 20, None,
                                    None) == B.EINVAL  # workspace not 256-byte aligned
+
+
+# --------------------------------------------------------------------------
+# FQCM and the bit-budget allocation: the library against the oracle, bit-exact
+# --------------------------------------------------------------------------
+
+def _unit(rng, E, r, d_out):
+    p = rng.standard_normal((E, r, d_out)).astype(np.float32)
+    return p / np.linalg.norm(p, axis=2, keepdims=True)
+
+
+@pytest.mark.parametrize("seed,E,r,d_out", [(1, 3, 40, 37), (2, 2, 64, 768)])
+def test_fqcm_eps_matches_oracle(B, orc, seed, E, r, d_out):
+    """Unit directions plus the special cases: a zero direction, a non-unit one past
+    fp16's scale range, one with a NaN."""
+    rng = np.random.default_rng(seed)
+    p = _unit(rng, E, r, d_out)
+    p[0, 0] = 0.0
+    p[0, 1] *= 1e6
+    p[0, 2, 3] = np.nan
+    got, ref = B.fqcm_eps(p), orc.fqcm_eps(p)
+    assert np.array_equal(got, ref, equal_nan=True)
+
+
+def test_fqcm_beta_matches_oracle(B, orc):
+    rng = np.random.default_rng(3)
+    T, K, E, r = 50, 4, 6, 33
+    Z = rng.standard_normal((T, r)).astype(np.float32)
+    ids = rng.integers(-1, E + 1, (T, K)).astype(np.int32)  # some ids out of range
+    g = rng.uniform(0, 1, (T, K)).astype(np.float32)
+    assert np.array_equal(B.fqcm_beta(Z, ids, g, E), orc.fqcm_beta(Z, ids, g, E))
+
+
+@pytest.mark.parametrize("seed", [4, 5])
+def test_allocate_widths_matches_oracle(B, orc, seed):
+    """The same inputs (seeded amplitudes, importances and distortions from the
+    oracle's own eps), several budgets from none to everything: identical widths
+    and total cost."""
+    rng = np.random.default_rng(seed)
+    E, r, d_out = 3, 50, 24
+    a = rng.lognormal(0, 0.5, (E, r)).astype(np.float32)
+    beta = rng.lognormal(0, 1.0, (E, r))
+    beta[0, :3] = 0.0
+    eps = orc.fqcm_eps(_unit(rng, E, r, d_out))
+    eps[1, 4, 2] = np.nan  # a component without a finite cost
+    for avg in (0.0, 0.5, 2.08, 3.0, 16.0):
+        budget = int(avg * E * r * d_out)
+        w, loss = B.allocate_widths(a, beta, eps, d_out, budget)
+        w_ref, loss_ref = orc.allocate_widths(a, beta, eps, d_out, budget)
+        assert np.array_equal(w, w_ref) and loss == loss_ref, avg
+        assert int(d_out * w.astype(np.int64).sum()) <= budget
+        assert w[1, 4] == 0
+
+
+def test_fqcm_argument_checks(B):
+    L = B.lib()
+    assert L.bitsmoe_fqcm_eps(None, 1, 1, 1, None) == B.EINVAL
+    assert L.bitsmoe_fqcm_beta(None, None, None, 1, 1, 1, 1, 256) == B.EINVAL
+    beta = np.full((1, 1), 7.0)
+    assert L.bitsmoe_fqcm_beta(None, None, None, 0, 1, 1, 1, beta.ctypes.data) == B.OK  # no tokens: zeros
+    assert beta[0, 0] == 0.0
+    assert L.bitsmoe_allocate_widths(None, None, None, 1, 1, 1, 0, None, None) == B.EINVAL
