@@ -44,38 +44,45 @@ static void parallel_ranges(int64_t n, F f) {
     for (auto& th : pool) th.join();
 }
 
-// The quantiser of the packed format on the host: q for element p at width b with
-// the fp16 scale value s: t = p / s and u = t + 2^(b-1) as separate fp32
-// operations, floor, clamp; q = 0 for a scale of 0 or one that is not finite.
-static uint32_t quantise_host(float p, int b, float s) {
-    if (!std::isfinite(s) || s <= 0.0f) return 0;  // a scale past fp16's range stores nothing
-    const float t = p / s;
-    const float u = t + (float)(1 << (b - 1));
-    const float f = std::floor(u);
-    const float qmax = (float)((1 << b) - 1);
-    if (f < 0.0f) return 0;
-    if (f > qmax) return (uint32_t)qmax;
-    return (uint32_t)f;
-}
-
-static double eps_of(const float* p, int d_out, int b, float m) {
-    double acc = 0.0;
-    float s = 0.0f;
-    if (b != 0 && b != 16) s = __half2float(__float2half_rn((2.0f * m) / (float)((1 << b) - 1)));
-    for (int i = 0; i < d_out; i++) {
-        double w;
-        if (b == 0) {
-            w = 0.0;
-        } else if (b == 16) {
-            w = (double)__half2float(__float2half_rn(p[i]));
-        } else {
-            const uint32_t q = quantise_host(p[i], b, s);
-            w = (double)s * ((double)q - (double)((1 << b) - 1) / 2.0);
-        }
-        const double d = (double)p[i] - w;
-        acc += d * d;
+// eps at every width of kWidthSet for one direction p (d_out elements, largest
+// magnitude m, all finite), in one pass over p: per element, every width's stored
+// value and squared error, each width's sum taken in element order in fp64.
+static void eps_all(const float* p, int d_out, float m, double* out) {
+    constexpr int kQ = 6;  // the widths with a scale: 1, 2, 3, 4, 6, 8
+    float s[kQ], half[kQ], qmax[kQ];
+    double mid[kQ], acc[kQ];
+    bool stores[kQ];
+    for (int j = 0; j < kQ; j++) {
+        const int b = kWidthSet[1 + j];
+        s[j] = __half2float(__float2half_rn((2.0f * m) / (float)((1 << b) - 1)));
+        stores[j] = std::isfinite(s[j]) && s[j] > 0.0f;  // else every q is 0
+        half[j] = (float)(1 << (b - 1));
+        qmax[j] = (float)((1 << b) - 1);
+        mid[j] = (double)((1 << b) - 1) / 2.0;
+        acc[j] = 0.0;
     }
-    return acc;
+    double acc0 = 0.0, acc16 = 0.0;
+    for (int i = 0; i < d_out; i++) {
+        const float x = p[i];
+        const double xd = (double)x;
+        acc0 += xd * xd;  // 0 bits: nothing stored
+        const double d16 = xd - (double)__half2float(__float2half_rn(x));  // 16 bits: fp16(p)
+        acc16 += d16 * d16;
+        for (int j = 0; j < kQ; j++) {
+            float q = 0.0f;
+            if (stores[j]) {
+                // t = x / s and u = t + 2^(b-1) as separate fp32 operations; for u >= 0
+                // the integer part is floor(u), and past the top level the clamp applies
+                const float u = x / s[j] + half[j];
+                q = u < 0.0f ? 0.0f : (float)(int)std::min(u, qmax[j]);
+            }
+            const double d = xd - (double)s[j] * ((double)q - mid[j]);
+            acc[j] += d * d;
+        }
+    }
+    out[0] = acc0;
+    for (int j = 0; j < kQ; j++) out[1 + j] = acc[j];
+    out[7] = acc16;
 }
 
 }  // namespace bitsmoe
@@ -94,7 +101,10 @@ BITSMOE_API int bitsmoe_fqcm_eps(const float* comps, int32_t E, int32_t r, int32
                 if (!std::isfinite(p[i])) bad = true;
                 m = std::max(m, std::fabs(p[i]));
             }
-            for (int wi = 0; wi < 8; wi++) out[wi] = bad ? NAN : eps_of(p, d_out, kWidthSet[wi], m);
+            if (bad)
+                for (int wi = 0; wi < 8; wi++) out[wi] = NAN;
+            else
+                eps_all(p, d_out, m, out);
         }
     });
     return BITSMOE_OK;
