@@ -28,7 +28,7 @@ __host__ __device__ constexpr uint32_t tc_idesc(int m, int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-// 2-D TMA tile load (no multicast) into shared memory, completing on an mbarrier.
+// 2-D TMA tile load into this CTA's shared memory alone, completing on an mbarrier.
 __device__ __forceinline__ void tc_tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
