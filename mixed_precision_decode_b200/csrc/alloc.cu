@@ -143,56 +143,89 @@ struct Seg {
 };
 }  // namespace
 
+// The lower convex hull of one component's (bits, loss) points from width 0, as
+// segments (out: up to 7), or none when its cost is not finite.
+static int hull_segments(int64_t c, double a, double beta, const double* eps8, int d_out, Seg* out) {
+    struct Pt {
+        int64_t bits;
+        double loss;
+        int wi;
+    };
+    const double imp = a * a * beta;
+    bool finite = std::isfinite(imp);
+    for (int wi = 0; wi < 8; wi++) finite = finite && std::isfinite(eps8[wi]);
+    if (!finite) return 0;  // a component without a finite cost keeps width 0
+    Pt hull[8];
+    int h = 0;
+    hull[h++] = {0, imp * eps8[0], 0};
+    for (int wi = 1; wi < 8; wi++) {
+        const Pt pt{(int64_t)d_out * kWidthSet[wi], imp * eps8[wi], wi};
+        if (pt.loss >= hull[h - 1].loss) continue;  // more bits and no less loss
+        while (h >= 2) {
+            const Pt& A = hull[h - 2];
+            const Pt& Bq = hull[h - 1];
+            if ((Bq.loss - A.loss) * (double)(pt.bits - A.bits) >= (pt.loss - A.loss) * (double)(Bq.bits - A.bits))
+                h--;
+            else
+                break;
+        }
+        hull[h++] = pt;
+    }
+    for (int s = 0; s + 1 < h; s++) {
+        const double gain = hull[s].loss - hull[s + 1].loss;
+        const int64_t cost = hull[s + 1].bits - hull[s].bits;
+        out[s] = {gain / (double)cost, c, s, cost, hull[s + 1].wi};
+    }
+    return h - 1;
+}
+
+static bool seg_before(const Seg& x, const Seg& y) {
+    if (x.eff != y.eff) return x.eff > y.eff;
+    if (x.c != y.c) return x.c < y.c;
+    return x.s < y.s;
+}
+
 BITSMOE_API int bitsmoe_allocate_widths(const float* amps, const double* beta, const double* eps, int32_t E,
                                         int32_t r, int32_t d_out, uint64_t budget_bits, uint8_t* widths,
                                         double* loss_out) {
     if (!amps || !beta || !eps || !widths || E < 1 || r < 1 || d_out < 1) return BITSMOE_EINVAL;
     const int64_t n = (int64_t)E * r;
-    // per component: the lower convex hull of (bits, loss) from width 0, as segments
-    std::vector<std::vector<Seg>> per((size_t)n);
+    // every component's hull segments into one array: count, offsets, then fill
+    std::vector<uint8_t> nseg((size_t)n);
     parallel_ranges(n, [&](int64_t c0, int64_t c1) {
-        struct Pt {
-            int64_t bits;
-            double loss;
-            int wi;
-        };
-        std::vector<Pt> hull;
-        for (int64_t c = c0; c < c1; c++) {
-            const double a = (double)amps[c];
-            const double imp = a * a * beta[c];
-            bool finite = std::isfinite(imp);
-            for (int wi = 0; wi < 8; wi++) finite = finite && std::isfinite(eps[(size_t)c * 8 + wi]);
-            if (!finite) continue;  // a component without a finite cost keeps width 0
-            hull.clear();
-            hull.push_back({0, imp * eps[(size_t)c * 8], 0});
-            for (int wi = 1; wi < 8; wi++) {
-                const Pt pt{(int64_t)d_out * kWidthSet[wi], imp * eps[(size_t)c * 8 + wi], wi};
-                if (pt.loss >= hull.back().loss) continue;  // more bits and no less loss
-                while (hull.size() >= 2) {
-                    const Pt& A = hull[hull.size() - 2];
-                    const Pt& Bq = hull.back();
-                    if ((Bq.loss - A.loss) * (double)(pt.bits - A.bits) >= (pt.loss - A.loss) * (double)(Bq.bits - A.bits))
-                        hull.pop_back();
-                    else
-                        break;
-                }
-                hull.push_back(pt);
-            }
-            std::vector<Seg>& out = per[(size_t)c];
-            for (size_t s = 0; s + 1 < hull.size(); s++) {
-                const double gain = hull[s].loss - hull[s + 1].loss;
-                const int64_t cost = hull[s + 1].bits - hull[s].bits;
-                out.push_back({gain / (double)cost, c, (int)s, cost, hull[s + 1].wi});
-            }
+        Seg tmp[7];
+        for (int64_t c = c0; c < c1; c++)
+            nseg[(size_t)c] = (uint8_t)hull_segments(c, (double)amps[c], beta[c], eps + (size_t)c * 8, d_out, tmp);
+    });
+    std::vector<int64_t> off((size_t)n + 1, 0);
+    for (int64_t c = 0; c < n; c++) off[(size_t)c + 1] = off[(size_t)c] + nseg[(size_t)c];
+    std::vector<Seg> segs((size_t)off[(size_t)n]);
+    parallel_ranges(n, [&](int64_t c0, int64_t c1) {
+        for (int64_t c = c0; c < c1; c++)
+            hull_segments(c, (double)amps[c], beta[c], eps + (size_t)c * 8, d_out, segs.data() + off[(size_t)c]);
+    });
+    // sorted by loss saved per bit (a strict total order: the result does not depend on
+    // how the sort is split): runs sorted on host threads, then merged pairwise
+    const int64_t m = (int64_t)segs.size();
+    const int64_t nt = std::max<int64_t>(1, std::min<int64_t>({(int64_t)std::thread::hardware_concurrency(), 16,
+                                                               m / 4096 + 1}));
+    std::vector<int64_t> bound((size_t)nt + 1);
+    for (int64_t t = 0; t <= nt; t++) bound[(size_t)t] = m * t / nt;
+    parallel_ranges(nt, [&](int64_t t0, int64_t t1) {
+        for (int64_t t = t0; t < t1; t++)
+            std::sort(segs.begin() + bound[(size_t)t], segs.begin() + bound[(size_t)t + 1], seg_before);
+    });
+    for (int64_t width = 1; width < nt; width *= 2) {
+        std::vector<std::thread> pool;
+        for (int64_t t = 0; t + width < nt; t += 2 * width) {
+            const int64_t a = bound[(size_t)t], mid = bound[(size_t)(t + width)],
+                          b = bound[(size_t)std::min(nt, t + 2 * width)];
+            pool.emplace_back([&segs, a, mid, b] {
+                std::inplace_merge(segs.begin() + a, segs.begin() + mid, segs.begin() + b, seg_before);
+            });
         }
-    });
-    std::vector<Seg> segs;
-    for (auto& v : per) segs.insert(segs.end(), v.begin(), v.end());
-    std::sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) {
-        if (x.eff != y.eff) return x.eff > y.eff;
-        if (x.c != y.c) return x.c < y.c;
-        return x.s < y.s;
-    });
+        for (auto& th : pool) th.join();
+    }
     std::vector<uint8_t> choice((size_t)n, 0);
     uint64_t used = 0;
     for (const Seg& sg : segs) {
