@@ -83,3 +83,27 @@ def test_reference_arm_uses_only_synth_and_oracle():
                                                                 fromlist=["CONFIGS"]).CONFIGS["tiny"], 4, 16)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_ffn_and_offline_byte_and_peak_formulas():
+    """The FFN line's bytes: each distinct routed expert's fp16 down matrix once, plus
+    the fp32 gate/up expert outputs, routing and output; the offline line's fp32
+    peak from the unit counts."""
+    import numpy as np
+    from mixed_precision_decode_b200 import synth
+    cfg = synth.CONFIGS["qwen_t1"]
+    ids = np.array([[3, 7, 3, 9, 1, 2, 4, 5]])  # expert 3 twice: read once
+    b = bench.down_bytes(cfg, ids, 1)
+    assert b["w_down"] == 7 * 2048 * 768 * 2
+    assert b["act"] == 2 * 1 * 8 * 768 * 4 + 1 * 8 * 8 + 1 * 2048 * 4
+    assert b["total"] == b["w_down"] + b["act"]
+    assert abs(bench.fp32_peak_tflops(1965.0) - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+
+
+def test_cli_modes_parse(monkeypatch):
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--ffn", "--ffn-two-calls", "--steps", "3"])
+    a = bench.parse()
+    assert a.ffn and a.ffn_two_calls and not a.ssd and a.steps == 3
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--ssd", "--fqcm", "--calib-tokens", "64"])
+    a = bench.parse()
+    assert a.ssd and a.fqcm and a.calib_tokens == 64 and not a.ffn
