@@ -105,3 +105,40 @@ def test_fqcm_argument_checks(B):
     assert L.bitsmoe_fqcm_beta(None, None, None, 0, 1, 1, 1, beta.ctypes.data) == B.OK  # no tokens: zeros
     assert beta[0, 0] == 0.0
     assert L.bitsmoe_allocate_widths(None, None, None, 1, 1, 1, 0, None, None) == B.EINVAL
+
+
+# --------------------------------------------------------------------------
+# property tests over random shapes, ties and budgets (bounded example counts)
+# --------------------------------------------------------------------------
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(E=st.integers(1, 4), r=st.integers(1, 24), seed=st.integers(0, 2 ** 31 - 1),
+       levels=st.integers(1, 6))
+def test_assign_widths_property(B, orc, E, r, seed, levels):
+    rng = np.random.default_rng(seed)
+    a = rng.integers(0, levels, (E, r)).astype(np.float32)  # few distinct values: many ties
+    order = tuple(int(b) for b in rng.permutation([0, 1, 2, 3, 4, 6, 8, 16])[:rng.integers(1, 9)])
+    cuts = np.sort(rng.integers(0, r + 1, len(order) - 1))
+    counts = np.diff(np.concatenate([[0], cuts, [r]])).astype(np.int32)
+    assert np.array_equal(B.assign_widths(a, order, counts), orc.assign_widths(a, order, counts))
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(E=st.integers(1, 3), r=st.integers(1, 20), d_out=st.integers(1, 40), seed=st.integers(0, 2 ** 31 - 1),
+       frac=st.floats(0.0, 1.2))
+def test_fqcm_and_allocation_property(B, orc, E, r, d_out, seed, frac):
+    rng = np.random.default_rng(seed)
+    p = rng.standard_normal((E, r, d_out)).astype(np.float32)
+    p[rng.random((E, r)) < 0.1] = 0.0  # some zero directions
+    eps = B.fqcm_eps(p)
+    assert np.array_equal(eps, orc.fqcm_eps(p), equal_nan=True)
+    a = rng.lognormal(0, 1, (E, r)).astype(np.float32)
+    beta = rng.lognormal(0, 1, (E, r)) * (rng.random((E, r)) > 0.2)
+    budget = int(frac * 16 * E * r * d_out)
+    w, loss = B.allocate_widths(a, beta, eps, d_out, budget)
+    w_ref, loss_ref = orc.allocate_widths(a, beta, eps, d_out, budget)
+    assert np.array_equal(w, w_ref) and loss == loss_ref
+    assert int(d_out * w.astype(np.int64).sum()) <= budget
